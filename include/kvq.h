@@ -1,0 +1,281 @@
+/*
+ * kvq.h -- C ABI of libkvq: attention over a block-quantized KV cache
+ * (Q8_0 keys, Q4_0 values) at long context, for NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages on quantized KV at long context):
+ *  "OSCAR2 KV Cache benchmark" (molayo1419.me), Compression Ratios table:
+ *      q8_0 costs 136 bytes per 128 elements (34-byte blocks of 32).
+ *  "Adaptive KV streaming lands on ROCm: Qwen3.8-27B at full 262k context ..."
+ *      (richland.au), "What shipped" and "Why it matters": the full KV history
+ *      stays in host RAM and a bounded working set is streamed to the GPU and
+ *      reused across layers; Q8_0 K + Q4_0 V costs 26,624 B/token for 16
+ *      attention layers of 4 KV heads x 256.
+ *  "Qwen 27B (IQ4_XS, Q8/Q4 KV) ... 262k context" (molayo1419.me), list of
+ *      improvements, "Online Log-Sum-Exp prefill & pipelined prefetch":
+ *      chunked prefill over streamed pages with online LSE accumulation, and
+ *      layer L+1's transfer overlapped with layer L's compute; speculative-
+ *      decoding paragraph: paged decode attention extended to the verify batch.
+ *  "Context window and KV cache" (localaiforum.com), "GQA" section: a few KV
+ *      heads are shared by many query heads; "levers" section: llama.cpp
+ *      quantizes the KV cache (q8_0 halves it, q4_0 quarters it).
+ *
+ * Conventions for every entry point
+ *  - The caller owns all memory.  Device buffers are passed as plain device
+ *    pointers; the library allocates no device memory.  kvq_layer structs and
+ *    arrays of them are read from HOST memory during the call only.
+ *  - Calls are asynchronous on the given stream (a cudaStream_t passed as
+ *    void*, NULL = the legacy default stream) and never synchronise, except
+ *    kvq_check.  Results are valid once the stream reaches that point.
+ *  - Arguments are validated before anything is launched.  On error nothing
+ *    is launched, the status says why and kvq_last_error() gives a
+ *    thread-local message.  A launch failure returns KVQ_ERR_CUDA.
+ *  - No call aborts, exits or traps.  Every device-side wait is bounded; a
+ *    wait that runs out records KVQ_ERR_TIMEOUT in a device status word that
+ *    kvq_check() reads and clears.
+ *  - fp16 values are passed as uint16_t bit patterns (IEEE binary16).
+ *
+ * Block formats (llama.cpp-style; the pages give sizes, these are the
+ * readings of the bit layout):
+ *  Q8_0, 34 B per 32 elements: fp16 d (little-endian) then int8 q[32];
+ *        x^ = d * q.  Quantized in fp32 without FMA: d = amax/127,
+ *        id = d ? 1/d : 0, q = roundf(x*id) (ties away from zero).
+ *  Q4_0, 18 B per 32 elements: fp16 d then 16 bytes; byte j holds element
+ *        j in the low nibble and element j+16 in the high nibble; x^ = d*(u-8).
+ *        m = the signed first element of largest |x|, d = m/-8,
+ *        id = d ? 1/d : 0, u = min(15, trunc(x*id + 8.5)).
+ *  Only fp16(d) is stored; the quantizer divides by the fp32 d.
+ *
+ * Cache layout of one layer (head-major, fixed):
+ *  K: [n_kv_heads][capacity][head_dim/32] Q8_0 blocks
+ *     -> one head-row of a token is head_dim/32*34 bytes (272 B at 256)
+ *  V: [n_kv_heads][capacity][head_dim/32] Q4_0 blocks
+ *     -> one head-row is head_dim/32*18 bytes (144 B at 256)
+ *  Head-rows of consecutive tokens of a head are contiguous, so a run of
+ *  tokens is one contiguous byte range.  Both base pointers must be 16-byte
+ *  aligned and capacity a multiple of 8: then every head starts on a 16-byte
+ *  boundary (8 head-rows are 272*(head_dim/32) or 144*(head_dim/32) bytes),
+ *  and so does every run of tokens that starts at a multiple of 8.
+ *  head_dim is a multiple of 32, at most 512.
+ *
+ * Attention (the plainest reading): query head g reads KV head
+ * g / (n_q_heads / n_kv_heads); s_j = scale * sum_i q_i k^_ij;
+ * o = sum_j exp(s_j - m) v^_j / l, lse = m + ln l (natural log), m the max
+ * over the complete visible scores, l = sum_j exp(s_j - m).  An empty key
+ * set gives o = 0 and lse = -inf.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvq_status {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size or shape              */
+    KVQ_ERR_ALIGNMENT = 2,    /* a pointer is not aligned as documented        */
+    KVQ_ERR_UNSUPPORTED = 3,  /* valid but not implemented (e.g. head_dim)     */
+    KVQ_ERR_CUDA = 4,         /* a CUDA runtime call or a launch failed        */
+    KVQ_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out            */
+    KVQ_ERR_COPY = 6,         /* a host<->device copy could not be enqueued    */
+    KVQ_ERR_WORKSPACE = 7     /* workspace missing or smaller than required    */
+} kvq_status;
+
+/* A cudaStream_t, passed as an opaque pointer so that this header needs no
+ * CUDA header.  NULL is the legacy default stream. */
+typedef void *kvq_stream;
+
+/* One attention layer of the cache.  All layers passed to one call must have
+ * the same n_kv_heads and head_dim. */
+typedef struct kvq_layer {
+    void *k;             /* K blocks, layout above (device memory, or pinned
+                            host memory for kvq_stream_decode's host_layers) */
+    void *v;             /* V blocks, layout above                           */
+    int64_t capacity;    /* tokens per head the two arrays hold              */
+    int32_t n_kv_heads;  /* KV heads (4 in the pages' hybrid model)          */
+    int32_t head_dim;    /* elements per head-row, a multiple of 32, <= 512  */
+} kvq_layer;
+
+/* Largest number of layers one call accepts (layer tables travel as kernel
+ * parameters). */
+#define KVQ_MAX_LAYERS 64
+/* Largest decode batch (query tokens per layer per call): the verify batch. */
+#define KVQ_MAX_DECODE_T 4
+
+/* ---------------------------------------------------------------------- */
+/* Quantize-on-append                                                      */
+/* ---------------------------------------------------------------------- */
+
+/* Quantize n fp32 values to Q8_0 blocks.
+ * Source: Compression Ratios table of the OSCAR2 page (34 B per 32 elements);
+ * the levers section of the KV-cache guide (q8_0 KV).
+ *  x      device, fp32[n], 4-byte aligned
+ *  blocks device, n/32 blocks of 34 bytes, written in order, 2-byte aligned
+ *  n      multiple of 32, >= 0 (0 launches nothing)
+ * Errors: INVALID_ARG (null pointer with n > 0, n % 32 != 0, n < 0),
+ *         ALIGNMENT (x not 4-byte or blocks not 2-byte aligned), CUDA. */
+kvq_status kvq_quantize_q8_0(const float *x, void *blocks, int64_t n, kvq_stream stream);
+
+/* Quantize n fp32 values to Q4_0 blocks (18 B per 32 elements).
+ * Source: 26,624 B/token in "Why it matters" of the ROCm streaming page
+ * implies 18 B per 32 V elements; the KV-cache guide's levers (q4_0 KV).
+ * Arguments and errors as kvq_quantize_q8_0. */
+kvq_status kvq_quantize_q4_0(const float *x, void *blocks, int64_t n, kvq_stream stream);
+
+/* Quantize-on-append of new K/V rows into rows [pos, pos+n_tok) of every KV
+ * head of n_layers layers (K -> Q8_0, V -> Q4_0).
+ * Source: the KV-cache guide's levers section (the KV cache is stored
+ * quantized); the Q8_0 K / Q4_0 V cache of the RX 9070 XT page.
+ *  layers  host array of n_layers kvq_layer (device caches)
+ *  k_new   device fp32 [n_layers][n_tok][n_kv_heads][head_dim], 16-B aligned
+ *  v_new   device fp32, same shape
+ *  pos     first row written; pos + n_tok <= capacity of every layer
+ * Errors: INVALID_ARG (nulls, n_layers outside [1, KVQ_MAX_LAYERS], n_tok < 1,
+ *         pos < 0, pos + n_tok > capacity, layers that differ in heads/dim,
+ *         capacity % 8 != 0), ALIGNMENT, UNSUPPORTED (head_dim not a multiple
+ *         of 32 or > 512), CUDA. */
+kvq_status kvq_append(const kvq_layer *layers, int n_layers, const float *k_new,
+                      const float *v_new, int64_t pos, int n_tok, kvq_stream stream);
+
+/* ---------------------------------------------------------------------- */
+/* Split-KV GQA decode attention                                           */
+/* ---------------------------------------------------------------------- */
+
+/* Decode attention of T query tokens per layer (T = 1 decode, T <= 4 a
+ * speculative verify batch) over the first n_kv keys of each layer, split
+ * into chunks of `chunk` keys; returns every chunk's partial (out, lse).
+ * Query token t sees keys j <= n_kv - T + t (n_kv counts the T new rows,
+ * which must already be appended).  Dequantization happens in registers;
+ * each chunk keeps an online softmax whose max covers complete scores.
+ * Source: speculative-decoding paragraph of the RX 9070 XT page (paged decode
+ * attention extended to the verify batch); "Known Issues Fixed" of the
+ * OSCAR2 page (max over the full KQ scores); GQA section of the KV-cache guide.
+ *  layers    host array of n_layers kvq_layer (device caches)
+ *  q         device fp16 bits [n_layers][T][n_q_heads][head_dim], 16-B aligned
+ *  n_q_heads multiple of n_kv_heads; n_q_heads/n_kv_heads * T <= 32
+ *  n_kv      keys per layer, T <= n_kv <= capacity
+ *  chunk     keys per chunk, a positive multiple of 64
+ *  scale     softmax scale applied to q.k (1/16 for head_dim 256)
+ *  out_part  device fp32 [n_layers][T][n_q_heads][n_chunks][head_dim], 16-B
+ *            aligned, n_chunks = ceil(n_kv / chunk); fully masked chunks get 0
+ *  lse_part  device fp32 [n_layers][T][n_q_heads][n_chunks]; -inf if masked
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (T > KVQ_MAX_DECODE_T, group
+ *         too large), CUDA. */
+kvq_status kvq_decode_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                           int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                           float *out_part, float *lse_part, kvq_stream stream);
+
+/* ---------------------------------------------------------------------- */
+/* LSE merge                                                               */
+/* ---------------------------------------------------------------------- */
+
+/* Merge per-chunk partials: lse = M + ln sum_c exp(lse_c - M) with
+ * M = max_c lse_c, out = sum_c exp(lse_c - lse) out_c; partials with
+ * lse_c = -inf are skipped; if every partial is -inf, out = 0, lse = -inf.
+ * Source: "Online Log-Sum-Exp prefill & pipelined prefetch" of the RX 9070 XT
+ * page (partials over pages combined through their log-sum-exp).
+ *  out_part device fp32 [rows][n_chunks][head_dim], 16-B aligned
+ *  lse_part device fp32 [rows][n_chunks]
+ *  out      device fp32 [rows][head_dim]; lse device fp32 [rows]
+ * Errors: INVALID_ARG (nulls, rows < 0, n_chunks < 1, head_dim % 4),
+ *         ALIGNMENT, CUDA. */
+kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t rows,
+                         int n_chunks, int head_dim, float *out, float *lse,
+                         kvq_stream stream);
+
+/* ---------------------------------------------------------------------- */
+/* Chunked prefill                                                         */
+/* ---------------------------------------------------------------------- */
+
+/* Prefill attention of T new query tokens per layer over n_cached + T keys
+ * (the T new rows must already be appended at rows [n_cached, n_cached+T));
+ * token t sees keys j <= n_cached + t.  Keys are processed page by page
+ * (`page` keys each) with an online LSE merge across pages; K and V tiles are
+ * dequantized on chip and the two contractions run on the tensor cores with
+ * fp32 accumulation.
+ * Source: "Online Log-Sum-Exp prefill & pipelined prefetch" of the RX 9070 XT
+ * page (chunked prefill over streamed pages with online LSE accumulation).
+ *  q         device fp16 bits [n_layers][T][n_q_heads][head_dim], 16-B aligned
+ *  n_cached  keys before the new rows; n_cached + T <= capacity
+ *  page      keys per page, a positive multiple of 128
+ *  out, lse  device fp32 [n_layers][T][n_q_heads][head_dim] and [...][n_q_heads]
+ *  page_out, page_lse  optional (both NULL or both set): per-page partials
+ *            [n_layers][T][n_q_heads][n_pages][head_dim] and [...][n_pages],
+ *            n_pages = ceil((n_cached + T) / page)
+ *  workspace device scratch of at least kvq_workspace_bytes(KVQ_OP_PREFILL,...)
+ *            bytes (may be NULL when that is 0), 256-B aligned
+ * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED (head_dim != 256 or
+ *         group size not dividing the 128-row tile), CUDA. */
+kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                            int n_q_heads, int T, int64_t n_cached, int page, float scale,
+                            float *out, float *lse, float *page_out, float *page_lse,
+                            void *workspace, size_t ws_bytes, kvq_stream stream);
+
+/* ---------------------------------------------------------------------- */
+/* Layer-pipelined host streaming                                          */
+/* ---------------------------------------------------------------------- */
+
+/* Decode attention with the cache in pinned host memory.  For each layer L
+ * the K and V rows [0, n_kv) of every head are copied with cudaMemcpyAsync on
+ * `copy` into device slot L % 2 while layer L-1 computes on `compute` in the
+ * other slot; then decode + merge of layer L run on `compute`.  Events order
+ * the two streams: the copy into a slot waits until the compute that last
+ * read it is done.  Results equal kvq_decode_attn + kvq_merge_lse on a
+ * resident cache bit for bit (same kernels, same data).
+ * Source: "Online Log-Sum-Exp prefill & pipelined prefetch" of the RX 9070 XT
+ * page (layer L+1's transfer overlapped with layer L's compute); "What
+ * shipped" of the ROCm streaming page (the whole KV history in host RAM, a
+ * bounded GPU working set reused across layers).
+ *  host_layers  host array of n_layers kvq_layer whose k/v are PINNED host
+ *               memory (cudaHostAlloc / cudaHostRegister)
+ *  dev_slots    host array of 2 kvq_layer (device memory), capacity >= n_kv,
+ *               same heads/dim as host_layers
+ *  q            device fp16 bits [n_layers][T][n_q_heads][head_dim]
+ *  out_part, lse_part  device scratch for ONE layer's partials:
+ *               [T][n_q_heads][n_chunks][head_dim] and [T][n_q_heads][n_chunks]
+ *  out, lse     device fp32 [n_layers][T][n_q_heads][head_dim], [...][n_q_heads]
+ *  compute, copy  two different streams
+ * The call enqueues everything and returns; `compute` is complete when all
+ * layers are.  Errors: those of kvq_decode_attn, plus COPY when a copy cannot
+ * be enqueued (nothing further is enqueued; work already enqueued completes). */
+kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_layers,
+                             const kvq_layer *dev_slots, const uint16_t *q, int n_q_heads,
+                             int T, int64_t n_kv, int chunk, float scale, float *out_part,
+                             float *lse_part, float *out, float *lse, kvq_stream compute,
+                             kvq_stream copy);
+
+/* ---------------------------------------------------------------------- */
+/* Housekeeping                                                            */
+/* ---------------------------------------------------------------------- */
+
+#define KVQ_OP_DECODE 1
+#define KVQ_OP_PREFILL 2
+
+/* Bytes of device workspace an operation needs (0 if none).
+ * KVQ_OP_DECODE: always 0.  KVQ_OP_PREFILL: n_layers, n_q_heads, T as the call.
+ * Returns (size_t)-1 for an unknown op. */
+size_t kvq_workspace_bytes(int op, int n_layers, int n_q_heads, int n_kv_heads, int T,
+                           int head_dim);
+
+/* Synchronise `stream`, then read and clear the device status word of the
+ * current device.  KVQ_OK, KVQ_ERR_TIMEOUT (a bounded wait ran out in some
+ * kernel since the last check) or KVQ_ERR_CUDA (an asynchronous CUDA error). */
+kvq_status kvq_check(kvq_stream stream);
+
+/* Static description of a status code (never NULL). */
+const char *kvq_status_string(kvq_status status);
+
+/* Thread-local detail of the last error returned on this thread ("" if none). */
+const char *kvq_last_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,390 @@
+// api.cu -- the extern "C" entry points of libkvq (declared in kvq.h):
+// argument validation, error reporting and dispatch to the kernels.
+//
+// Every entry point validates all of its arguments before it launches
+// anything; on an error it returns the status and leaves a thread-local
+// message for kvq_last_error().  Nothing here synchronises except kvq_check.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <cmath>
+
+#include "common.cuh"
+
+namespace kvq {
+
+// Status word written by kernels whose bounded waits run out.  Host code
+// reaches it through the address cudaGetSymbolAddress reports for the
+// current device (cached per device).
+static __device__ unsigned int g_status_word;
+
+static thread_local char t_err[512];
+
+kvq_status set_error(kvq_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_err, sizeof(t_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+kvq_status check_launch(const char *what)
+{
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return set_error(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return KVQ_OK;
+}
+
+kvq_status status_word(unsigned int **out)
+{
+    constexpr int MAX_DEV = 64;
+    static unsigned int *cache[MAX_DEV] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV)
+        return set_error(KVQ_ERR_CUDA, "no current CUDA device");
+    if (!cache[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
+        if (e != cudaSuccess)
+            return set_error(KVQ_ERR_CUDA, "status word: %s", cudaGetErrorString(e));
+        cache[dev] = static_cast<unsigned int *>(p);
+    }
+    *out = cache[dev];
+    return KVQ_OK;
+}
+
+// ---- validation helpers ---------------------------------------------------
+
+static kvq_status check_layers(const kvq_layer *layers, int n_layers, const char *fn)
+{
+    if (!layers)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: layers is NULL", fn);
+    if (n_layers < 1 || n_layers > KVQ_MAX_LAYERS)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_layers=%d outside [1, %d]", fn, n_layers,
+                         KVQ_MAX_LAYERS);
+    const int H = layers[0].n_kv_heads, D = layers[0].head_dim;
+    if (H < 1)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_kv_heads=%d", fn, H);
+    if (D < QK || D % QK != 0)
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: head_dim=%d is not a positive multiple of 32",
+                         fn, D);
+    if (D > 512)
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: head_dim=%d > 512", fn, D);
+    for (int l = 0; l < n_layers; ++l) {
+        const kvq_layer &L = layers[l];
+        if (!L.k || !L.v)
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: layer %d has a NULL cache pointer", fn, l);
+        if (L.n_kv_heads != H || L.head_dim != D)
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: layer %d differs in heads/head_dim", fn, l);
+        if (L.capacity < 1 || L.capacity % 8 != 0)
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: layer %d capacity=%lld not a positive "
+                             "multiple of 8", fn, l, (long long)L.capacity);
+        if (!aligned(L.k, 16) || !aligned(L.v, 16))
+            return set_error(KVQ_ERR_ALIGNMENT, "%s: layer %d cache not 16-byte aligned", fn, l);
+    }
+    return KVQ_OK;
+}
+
+template <typename P>
+static kvq_status need(const P *p, uintptr_t align, const char *name, const char *fn)
+{
+    if (!p)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: %s is NULL", fn, name);
+    if (!aligned(p, align))
+        return set_error(KVQ_ERR_ALIGNMENT, "%s: %s not %d-byte aligned", fn, name, (int)align);
+    return KVQ_OK;
+}
+
+#define KVQ_TRY(expr)                      \
+    do {                                   \
+        const kvq_status _s = (expr);      \
+        if (_s != KVQ_OK)                  \
+            return _s;                     \
+    } while (0)
+
+static void fill_table(const kvq_layer *layers, int n, LayerTable &t)
+{
+    for (int l = 0; l < KVQ_MAX_LAYERS; ++l) {
+        t.k[l] = l < n ? static_cast<const uint8_t *>(layers[l].k) : nullptr;
+        t.v[l] = l < n ? static_cast<const uint8_t *>(layers[l].v) : nullptr;
+        t.cap[l] = l < n ? layers[l].capacity : 0;
+    }
+}
+
+// Shared by kvq_decode_attn and kvq_stream_decode.
+kvq_status validate_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                           int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                           const float *out_part, const float *lse_part, const char *fn)
+{
+    KVQ_TRY(check_layers(layers, n_layers, fn));
+    KVQ_TRY(need(q, 16, "q", fn));
+    KVQ_TRY(need(out_part, 16, "out_part", fn));
+    KVQ_TRY(need(lse_part, 4, "lse_part", fn));
+    const int H = layers[0].n_kv_heads;
+    if (n_q_heads < 1 || n_q_heads % H != 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_q_heads=%d not a multiple of n_kv_heads=%d",
+                         fn, n_q_heads, H);
+    if (T < 1)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: T=%d < 1", fn, T);
+    if (T > KVQ_MAX_DECODE_T)
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: T=%d > %d", fn, T, KVQ_MAX_DECODE_T);
+    if ((n_q_heads / H) * T > 32)
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: group*T=%d > 32 rows", fn,
+                         (n_q_heads / H) * T);
+    if (chunk < 64 || chunk % 64 != 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: chunk=%d not a positive multiple of 64", fn,
+                         chunk);
+    if (n_kv < T)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_kv=%lld < T=%d", fn, (long long)n_kv, T);
+    for (int l = 0; l < n_layers; ++l)
+        if (n_kv > layers[l].capacity)
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: n_kv=%lld > capacity of layer %d", fn,
+                             (long long)n_kv, l);
+    if (!std::isfinite(scale))
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+    if ((n_kv + chunk - 1) / chunk > (1ll << 30))
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: too many chunks", fn);
+    return KVQ_OK;
+}
+
+kvq_status enqueue_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                          int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                          float *out_part, float *lse_part, cudaStream_t s)
+{
+    DecodeArgs a;
+    fill_table(layers, n_layers, a.layers);
+    a.n_layers = n_layers;
+    a.n_kv_heads = layers[0].n_kv_heads;
+    a.head_dim = layers[0].head_dim;
+    a.n_q_heads = n_q_heads;
+    a.T = T;
+    a.n_kv = n_kv;
+    a.chunk = chunk;
+    a.scale = scale;
+    a.q = reinterpret_cast<const __half *>(q);
+    a.out_part = out_part;
+    a.lse_part = lse_part;
+    KVQ_TRY(status_word(&a.status));
+    if (!launch_decode(a, s))
+        return set_error(KVQ_ERR_UNSUPPORTED, "kvq_decode_attn: no kernel for this shape");
+    return check_launch("kvq_decode_attn");
+}
+
+kvq_status validate_merge(const float *out_part, const float *lse_part, int64_t rows,
+                          int n_chunks, int head_dim, const float *out, const float *lse,
+                          const char *fn)
+{
+    KVQ_TRY(need(out_part, 16, "out_part", fn));
+    KVQ_TRY(need(lse_part, 4, "lse_part", fn));
+    KVQ_TRY(need(out, 16, "out", fn));
+    KVQ_TRY(need(lse, 4, "lse", fn));
+    if (rows < 0 || rows >= (1ll << 31))
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: rows=%lld", fn, (long long)rows);
+    if (n_chunks < 1)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_chunks=%d < 1", fn, n_chunks);
+    if (head_dim < 4 || head_dim % 4 != 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: head_dim=%d not a positive multiple of 4", fn,
+                         head_dim);
+    return KVQ_OK;
+}
+
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+kvq_status kvq_quantize_q8_0(const float *x, void *blocks, int64_t n, kvq_stream stream)
+{
+    const char *fn = "kvq_quantize_q8_0";
+    if (n < 0 || n % QK != 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n=%lld not a non-negative multiple of 32", fn,
+                         (long long)n);
+    if (n == 0)
+        return KVQ_OK;
+    KVQ_TRY(need(x, 4, "x", fn));
+    KVQ_TRY(need(static_cast<const uint8_t *>(blocks), 2, "blocks", fn));
+    launch_quantize_q8_0(x, static_cast<uint8_t *>(blocks), n, as_stream(stream));
+    return check_launch(fn);
+}
+
+kvq_status kvq_quantize_q4_0(const float *x, void *blocks, int64_t n, kvq_stream stream)
+{
+    const char *fn = "kvq_quantize_q4_0";
+    if (n < 0 || n % QK != 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n=%lld not a non-negative multiple of 32", fn,
+                         (long long)n);
+    if (n == 0)
+        return KVQ_OK;
+    KVQ_TRY(need(x, 4, "x", fn));
+    KVQ_TRY(need(static_cast<const uint8_t *>(blocks), 2, "blocks", fn));
+    launch_quantize_q4_0(x, static_cast<uint8_t *>(blocks), n, as_stream(stream));
+    return check_launch(fn);
+}
+
+kvq_status kvq_append(const kvq_layer *layers, int n_layers, const float *k_new,
+                      const float *v_new, int64_t pos, int n_tok, kvq_stream stream)
+{
+    const char *fn = "kvq_append";
+    KVQ_TRY(check_layers(layers, n_layers, fn));
+    KVQ_TRY(need(k_new, 16, "k_new", fn));
+    KVQ_TRY(need(v_new, 16, "v_new", fn));
+    if (n_tok < 1)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_tok=%d < 1", fn, n_tok);
+    if (pos < 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: pos=%lld < 0", fn, (long long)pos);
+    for (int l = 0; l < n_layers; ++l)
+        if (pos + n_tok > layers[l].capacity)
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: rows [%lld, %lld) exceed capacity of "
+                             "layer %d", fn, (long long)pos, (long long)(pos + n_tok), l);
+    const int H = layers[0].n_kv_heads, D = layers[0].head_dim;
+    if ((int64_t)n_layers * n_tok * H >= (1ll << 31))
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: too many rows in one call", fn);
+    if (2 * (D / QK) * 32 > 1024)
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: head_dim=%d", fn, D);
+    MutLayerTable t;
+    for (int l = 0; l < KVQ_MAX_LAYERS; ++l) {
+        t.k[l] = l < n_layers ? static_cast<uint8_t *>(layers[l].k) : nullptr;
+        t.v[l] = l < n_layers ? static_cast<uint8_t *>(layers[l].v) : nullptr;
+        t.cap[l] = l < n_layers ? layers[l].capacity : 0;
+    }
+    launch_append(t, n_layers, H, D, k_new, v_new, pos, n_tok, as_stream(stream));
+    return check_launch(fn);
+}
+
+kvq_status kvq_decode_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                           int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                           float *out_part, float *lse_part, kvq_stream stream)
+{
+    KVQ_TRY(validate_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
+                            lse_part, "kvq_decode_attn"));
+    return enqueue_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
+                          lse_part, as_stream(stream));
+}
+
+kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t rows,
+                         int n_chunks, int head_dim, float *out, float *lse, kvq_stream stream)
+{
+    const char *fn = "kvq_merge_lse";
+    KVQ_TRY(validate_merge(out_part, lse_part, rows, n_chunks, head_dim, out, lse, fn));
+    launch_merge_lse(out_part, lse_part, rows, n_chunks, head_dim, out, lse, as_stream(stream));
+    return check_launch(fn);
+}
+
+kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                            int n_q_heads, int T, int64_t n_cached, int page, float scale,
+                            float *out, float *lse, float *page_out, float *page_lse,
+                            void *workspace, size_t ws_bytes, kvq_stream stream)
+{
+    const char *fn = "kvq_prefill_attn";
+    KVQ_TRY(check_layers(layers, n_layers, fn));
+    KVQ_TRY(need(q, 16, "q", fn));
+    KVQ_TRY(need(out, 16, "out", fn));
+    KVQ_TRY(need(lse, 4, "lse", fn));
+    if ((page_out == nullptr) != (page_lse == nullptr))
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: page_out and page_lse must both be set or "
+                         "both be NULL", fn);
+    if (page_out) {
+        KVQ_TRY(need(page_out, 16, "page_out", fn));
+        KVQ_TRY(need(page_lse, 4, "page_lse", fn));
+    }
+    const int H = layers[0].n_kv_heads, D = layers[0].head_dim;
+    if (n_q_heads < 1 || n_q_heads % H != 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_q_heads=%d not a multiple of n_kv_heads=%d",
+                         fn, n_q_heads, H);
+    if (T < 1)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: T=%d < 1", fn, T);
+    if (n_cached < 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_cached < 0", fn);
+    if (page < 128 || page % 128 != 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: page=%d not a positive multiple of 128", fn,
+                         page);
+    for (int l = 0; l < n_layers; ++l)
+        if (n_cached + T > layers[l].capacity)
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: n_cached + T exceeds capacity of layer %d",
+                             fn, l);
+    if (!std::isfinite(scale))
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+    if (!prefill_supported(n_q_heads, H, D))
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: head_dim=%d, group=%d not supported", fn, D,
+                         n_q_heads / H);
+    const size_t ws = prefill_workspace_bytes(n_layers, n_q_heads, H, T, D);
+    if (ws > 0 && (workspace == nullptr || ws_bytes < ws))
+        return set_error(KVQ_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn,
+                         ws, workspace ? ws_bytes : (size_t)0);
+    if (ws > 0 && !aligned(workspace, 256))
+        return set_error(KVQ_ERR_ALIGNMENT, "%s: workspace not 256-byte aligned", fn);
+    PrefillArgs a;
+    fill_table(layers, n_layers, a.layers);
+    a.n_layers = n_layers;
+    a.n_kv_heads = H;
+    a.head_dim = D;
+    a.n_q_heads = n_q_heads;
+    a.T = T;
+    a.n_cached = n_cached;
+    a.page = page;
+    a.scale = scale;
+    a.q = reinterpret_cast<const __half *>(q);
+    a.out = out;
+    a.lse = lse;
+    a.page_out = page_out;
+    a.page_lse = page_lse;
+    a.workspace = workspace;
+    a.ws_bytes = ws_bytes;
+    KVQ_TRY(status_word(&a.status));
+    launch_prefill(a, as_stream(stream));
+    return check_launch(fn);
+}
+
+size_t kvq_workspace_bytes(int op, int n_layers, int n_q_heads, int n_kv_heads, int T,
+                           int head_dim)
+{
+    if (op == KVQ_OP_DECODE)
+        return 0;
+    if (op == KVQ_OP_PREFILL)
+        return prefill_workspace_bytes(n_layers, n_q_heads, n_kv_heads, T, head_dim);
+    return (size_t)-1;
+}
+
+kvq_status kvq_check(kvq_stream stream)
+{
+    cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+    if (e != cudaSuccess)
+        return set_error(KVQ_ERR_CUDA, "kvq_check: %s", cudaGetErrorString(e));
+    unsigned int *w = nullptr;
+    KVQ_TRY(status_word(&w));
+    unsigned int v = 0;
+    e = cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess)
+        return set_error(KVQ_ERR_CUDA, "kvq_check: %s", cudaGetErrorString(e));
+    if (v != 0) {
+        const unsigned int zero = 0;
+        cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        if (v & STATUS_TIMEOUT)
+            return set_error(KVQ_ERR_TIMEOUT, "kvq_check: a bounded device wait ran out");
+    }
+    return KVQ_OK;
+}
+
+const char *kvq_status_string(kvq_status s)
+{
+    switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_ALIGNMENT: return "misaligned pointer";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported shape";
+    case KVQ_ERR_CUDA: return "CUDA error";
+    case KVQ_ERR_TIMEOUT: return "device wait timed out";
+    case KVQ_ERR_COPY: return "copy could not be enqueued";
+    case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+const char *kvq_last_error(void) { return t_err; }
+
+int kvq_version(void) { return 100; }
+
+}  // extern "C"

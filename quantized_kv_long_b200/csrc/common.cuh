@@ -1,0 +1,90 @@
+// common.cuh -- shared definitions of the CUDA library (not of the oracle).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int QK = 32;           // elements per quantization block
+constexpr int Q8_0_BYTES = 34;   // fp16 d + 32 x int8
+constexpr int Q4_0_BYTES = 18;   // fp16 d + 16 bytes of nibbles
+
+__host__ __device__ inline int64_t k_row_bytes(int head_dim) { return (int64_t)(head_dim / QK) * Q8_0_BYTES; }
+__host__ __device__ inline int64_t v_row_bytes(int head_dim) { return (int64_t)(head_dim / QK) * Q4_0_BYTES; }
+
+// Layer table passed by value as a kernel parameter.
+struct LayerTable {
+    const uint8_t *k[KVQ_MAX_LAYERS];
+    const uint8_t *v[KVQ_MAX_LAYERS];
+    int64_t cap[KVQ_MAX_LAYERS];
+};
+
+struct MutLayerTable {
+    uint8_t *k[KVQ_MAX_LAYERS];
+    uint8_t *v[KVQ_MAX_LAYERS];
+    int64_t cap[KVQ_MAX_LAYERS];
+};
+
+// Device status word: bit flags set by kernels whose bounded waits ran out.
+// Kernels receive its address as a parameter (see status_word()).
+constexpr unsigned STATUS_TIMEOUT = 1u;
+
+__device__ __forceinline__ void report_timeout(unsigned int *status)
+{
+    atomicOr(status, STATUS_TIMEOUT);
+}
+
+// Bounded spin limit for any device-side wait (iterations of a try_wait loop).
+constexpr long long SPIN_LIMIT = 1ll << 26;
+
+// ---- error plumbing (host) ------------------------------------------------
+kvq_status set_error(kvq_status s, const char *fmt, ...);
+kvq_status check_launch(const char *what);
+kvq_status status_word(unsigned int **out);  // address of the current device's word
+
+inline bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+inline cudaStream_t as_stream(kvq_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ---- launchers (host, internal) -------------------------------------------
+void launch_quantize_q8_0(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s);
+void launch_quantize_q4_0(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s);
+void launch_append(const MutLayerTable &t, int n_layers, int n_kv_heads, int head_dim,
+                   const float *k_new, const float *v_new, int64_t pos, int n_tok,
+                   cudaStream_t s);
+void launch_merge_lse(const float *out_part, const float *lse_part, int64_t rows, int n_chunks,
+                      int head_dim, float *out, float *lse, cudaStream_t s);
+
+struct DecodeArgs {
+    LayerTable layers;
+    int n_layers, n_kv_heads, head_dim, n_q_heads, T;
+    int64_t n_kv;
+    int chunk;
+    float scale;
+    const __half *q;
+    float *out_part, *lse_part;
+    unsigned int *status;  // device status word (bounded waits that ran out)
+};
+// Returns false (and launches nothing) if no kernel supports the shape.
+bool launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+struct PrefillArgs {
+    LayerTable layers;
+    int n_layers, n_kv_heads, head_dim, n_q_heads, T;
+    int64_t n_cached;
+    int page;
+    float scale;
+    const __half *q;
+    float *out, *lse, *page_out, *page_lse;
+    void *workspace;
+    size_t ws_bytes;
+    unsigned int *status;
+};
+size_t prefill_workspace_bytes(int n_layers, int n_q_heads, int n_kv_heads, int T, int head_dim);
+bool prefill_supported(int n_q_heads, int n_kv_heads, int head_dim);
+void launch_prefill(const PrefillArgs &a, cudaStream_t s);
+
+}  // namespace kvq

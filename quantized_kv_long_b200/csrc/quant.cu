@@ -1,0 +1,154 @@
+// quant.cu -- quantize-on-append: fp32 rows -> Q8_0 (K) and Q4_0 (V) blocks.
+//
+// One warp quantizes one 32-element block: lane i holds element i, the block
+// maximum comes from warp shuffles, and every arithmetic step is an explicitly
+// rounded fp32 operation (__fdiv_rn, __fmul_rn, __fadd_rn) so that no
+// multiply-add is contracted and the blocks are bit-identical to any other
+// IEEE implementation of the same definition.
+//
+// Definitions (llama.cpp-style blocks; sizes from the "Compression Ratios"
+// table of the OSCAR2 KV-cache benchmark page and the 26,624 B/token of "Why
+// it matters" on the ROCm KV-streaming page; the rules are the plainest
+// reading of "d = amax/127, int8 round-to-nearest" and "d = max/-8, nibbles
+// q+8 clamped to 0..15"):
+//   Q8_0: d = amax/127; id = d ? 1/d : 0; q = roundf(x*id)  (ties away from 0)
+//   Q4_0: m = signed first max-|x| element (+0 if the block is all zeros);
+//         d = m/-8; id = d ? 1/d : 0; u = min(15, trunc(x*id + 8.5));
+//         byte j = u_j | u_{j+16} << 4
+//   fp16(d) stored first, little-endian.
+#include "common.cuh"
+
+namespace kvq {
+
+// The fp16 scale is converted by every lane (outside any lane-divergent
+// branch) and lane 0 stores it as one 16-bit word; blocks start at even byte
+// offsets (34*b, 18*b) of a 2-byte aligned buffer.  A byte-wise store of a
+// value converted inside the lane-0 branch was observed to write 0 into the
+// low byte on sm_100a; the bit-exact tests against the oracle caught it.
+__device__ __forceinline__ unsigned short d_bits(float d)
+{
+    return __half_as_ushort(__float2half_rn(d));
+}
+
+__device__ __forceinline__ void store_d(uint8_t *blk, unsigned short h)
+{
+    *reinterpret_cast<unsigned short *>(blk) = h;
+}
+
+// Lane `lane` holds x = element `lane` of the block that starts at `blk`.
+__device__ __forceinline__ void warp_quant_q8_0(float x, uint8_t *blk, int lane)
+{
+    float amax = fabsf(x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float d = __fdiv_rn(amax, 127.0f);
+    const float id = (d != 0.0f) ? __fdiv_rn(1.0f, d) : 0.0f;
+    const int q = (int)roundf(__fmul_rn(x, id));
+    const unsigned short h = d_bits(d);
+    blk[2 + lane] = (uint8_t)(int8_t)q;
+    if (lane == 0)
+        store_d(blk, h);
+}
+
+__device__ __forceinline__ void warp_quant_q4_0(float x, uint8_t *blk, int lane)
+{
+    // first index of the largest |x|: larger magnitude wins, ties go to the lower lane
+    float a = fabsf(x);
+    int idx = lane;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float a2 = __shfl_xor_sync(0xffffffffu, a, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
+        if (a2 > a || (a2 == a && i2 < idx)) {
+            a = a2;
+            idx = i2;
+        }
+    }
+    const float xm = __shfl_sync(0xffffffffu, x, idx);
+    const float m = (a > 0.0f) ? xm : 0.0f;  // an all-zero block keeps m = +0
+    const float d = __fdiv_rn(m, -8.0f);
+    const float id = (d != 0.0f) ? __fdiv_rn(1.0f, d) : 0.0f;
+    const float s = __fadd_rn(__fmul_rn(x, id), 8.5f);
+    int u = (int)truncf(s);
+    u = u > 15 ? 15 : u;
+    const int u_hi = __shfl_down_sync(0xffffffffu, u, 16);
+    const unsigned short h = d_bits(d);
+    if (lane < 16)
+        blk[2 + lane] = (uint8_t)(u | (u_hi << 4));
+    if (lane == 0)
+        store_d(blk, h);
+}
+
+template <bool Q8>
+__global__ void quantize_kernel(const float *__restrict__ x, uint8_t *__restrict__ blocks,
+                                int64_t n_blocks)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t b = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); b < n_blocks;
+         b += warps) {
+        const float v = x[b * QK + lane];
+        if (Q8)
+            warp_quant_q8_0(v, blocks + b * Q8_0_BYTES, lane);
+        else
+            warp_quant_q4_0(v, blocks + b * Q4_0_BYTES, lane);
+    }
+}
+
+static int quant_grid(int64_t n_blocks)
+{
+    const int64_t per_cta = 8;  // 256 threads
+    int64_t g = (n_blocks + per_cta - 1) / per_cta;
+    const int64_t cap = 148 * 16;
+    return (int)(g < cap ? (g > 0 ? g : 1) : cap);
+}
+
+void launch_quantize_q8_0(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s)
+{
+    const int64_t nb = n / QK;
+    quantize_kernel<true><<<quant_grid(nb), 256, 0, s>>>(x, blocks, nb);
+}
+
+void launch_quantize_q4_0(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s)
+{
+    const int64_t nb = n / QK;
+    quantize_kernel<false><<<quant_grid(nb), 256, 0, s>>>(x, blocks, nb);
+}
+
+// Append: one CTA per (layer, token, kv head); warps [0, nb) quantize the K
+// blocks of the head-row, warps [nb, 2 nb) the V blocks (nb = head_dim / 32).
+__global__ void append_kernel(MutLayerTable t, int n_kv_heads, int head_dim,
+                              const float *__restrict__ k_new, const float *__restrict__ v_new,
+                              int64_t pos, int n_tok)
+{
+    const int h = blockIdx.x % n_kv_heads;
+    const int tok = (blockIdx.x / n_kv_heads) % n_tok;
+    const int layer = blockIdx.x / (n_kv_heads * n_tok);
+    const int nb = head_dim / QK;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool is_v = w >= nb;
+    const int b = is_v ? w - nb : w;
+    const size_t src = (((size_t)layer * n_tok + tok) * n_kv_heads + h) * head_dim + (size_t)b * QK;
+    const int64_t row = (int64_t)h * t.cap[layer] + pos + tok;
+    if (!is_v) {
+        uint8_t *dst = t.k[layer] + row * k_row_bytes(head_dim) + (int64_t)b * Q8_0_BYTES;
+        warp_quant_q8_0(k_new[src + lane], dst, lane);
+    } else {
+        uint8_t *dst = t.v[layer] + row * v_row_bytes(head_dim) + (int64_t)b * Q4_0_BYTES;
+        warp_quant_q4_0(v_new[src + lane], dst, lane);
+    }
+}
+
+void launch_append(const MutLayerTable &t, int n_layers, int n_kv_heads, int head_dim,
+                   const float *k_new, const float *v_new, int64_t pos, int n_tok,
+                   cudaStream_t s)
+{
+    const int64_t ctas = (int64_t)n_layers * n_tok * n_kv_heads;
+    const int threads = 2 * (head_dim / QK) * 32;
+    // grid.x is at most 2^31-1; n_tok is an int and n_layers <= 64, heads small
+    append_kernel<<<(unsigned)ctas, threads, 0, s>>>(t, n_kv_heads, head_dim, k_new, v_new, pos,
+                                                     n_tok);
+}
+
+}  // namespace kvq

@@ -1,0 +1,58 @@
+"""Helpers shared by the GPU parity tests: caches built on both sides from
+the same seeded inputs, and the tolerance checks.
+
+Tolerances (written here once, used by every attention parity test):
+  * out: max |gpu - oracle| <= 2e-3 (absolute, fp32 output vs fp64 oracle);
+  * lse: |gpu - oracle| <= 1e-4 * max(|oracle|, 1) (relative, natural log);
+  * quantized blocks: bit-exact.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from quantized_kv_long_b200 import workload as wl
+
+OUT_ATOL = 2e-3
+LSE_RTOL = 1e-4
+
+
+def assert_attn_close(out, lse, ref_out, ref_lse, what=""):
+    out = np.asarray(out, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    ref_out = np.asarray(ref_out)
+    ref_lse = np.asarray(ref_lse)
+    masked = ref_lse == -np.inf
+    assert (lse[masked] == -np.inf).all(), f"{what}: masked partials must have lse = -inf"
+    assert (out[masked] == 0).all(), f"{what}: masked partials must be 0"
+    live = ~masked
+    if live.any():
+        err = np.abs(out[live] - ref_out[live]).max()
+        assert err <= OUT_ATOL, f"{what}: out max-abs error {err:.3e} > {OUT_ATOL}"
+        den = np.maximum(np.abs(ref_lse[live]), 1.0)
+        lerr = (np.abs(lse[live] - ref_lse[live]) / den).max()
+        assert lerr <= LSE_RTOL, f"{what}: lse relative error {lerr:.3e} > {LSE_RTOL}"
+
+
+def fill_both(w: wl.Workload, layers, n_rows: int, capacity: int, device="cuda"):
+    """Quantize rows [0, n_rows) of the given layers on the GPU (through
+    kvq_append) and on the CPU (oracle).  Returns (gpu cache, oracle caches)."""
+    from quantized_kv_long_b200 import kvq
+    cache = kvq.QuantizedKVCache(len(layers), w.n_kv_heads, w.head_dim, capacity, device=device)
+    orc = []
+    for i, l in enumerate(layers):
+        k = wl.kv_rows(w, l, 0, 0, n_rows)
+        v = wl.kv_rows(w, l, 1, 0, n_rows)
+        kt = torch.from_numpy(k).to(device)
+        vt = torch.from_numpy(v).to(device)
+        kvq.kvq_append(cache.layer(i), kt, vt, 0, n_rows)
+        kc, vc = oracle.empty_cache(w.n_kv_heads, w.head_dim, capacity)
+        oracle.append(kc, vc, k, v, 0)
+        orc.append((kc, vc))
+    torch.cuda.synchronize()
+    return cache, orc
+
+
+def q_all(w: wl.Workload, layers, T: int | None = None) -> np.ndarray:
+    return np.stack([wl.q_rows(w, l, T) for l in layers])

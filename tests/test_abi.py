@@ -1,0 +1,146 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects bad arguments with the documented status before launching anything
+(these calls make no CUDA compute call, so they run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from quantized_kv_long_b200 import build
+    build.build()
+    from quantized_kv_long_b200 import kvq as m
+    return m
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(kvq):
+    names = _declared()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(kvq.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(kvq.EXPORTED)
+
+
+def test_status_strings(kvq):
+    for s in range(8):
+        assert kvq.kvq_status_string(s) not in ("", "unknown status")
+    assert kvq.kvq_status_string(99) == "unknown status"
+    assert kvq.kvq_version() >= 100
+
+
+def _raises(kvq, status, fn, *a, **k):
+    with pytest.raises(kvq.KvqError) as e:
+        fn(*a, **k)
+    assert e.value.status == status, str(e.value)
+    assert kvq.kvq_last_error()
+
+
+A = 1 << 20  # a 16-byte aligned fake device address: never dereferenced here
+
+
+def _layer(kvq, **kw):
+    d = dict(k=A, v=A, capacity=1024, n_kv_heads=4, head_dim=256)
+    d.update(kw)
+    return kvq.kvq_layer(d["k"], d["v"], d["capacity"], d["n_kv_heads"], d["head_dim"])
+
+
+def test_quantize_validation(kvq):
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_quantize_q8_0, A, A, 33, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_quantize_q4_0, A, A, -32, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_quantize_q8_0, None, A, 64, 0)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_quantize_q4_0, A + 2, A, 64, 0)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_quantize_q8_0, A, A + 1, 64, 0)
+    kvq.kvq_quantize_q8_0(None, None, 0, 0)  # n == 0 launches nothing
+
+
+def test_append_validation(kvq):
+    L = _layer(kvq)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, L, None, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_append, L, A + 4, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, L, A, A, 1020, 5, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, L, A, A, -1, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, L, A, A, 0, 0, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, _layer(kvq, capacity=1020), A, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_append, _layer(kvq, k=A + 8), A, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_UNSUPPORTED, kvq.kvq_append, _layer(kvq, head_dim=48), A, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_UNSUPPORTED, kvq.kvq_append, _layer(kvq, head_dim=1024), A, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, [L, _layer(kvq, n_kv_heads=2)], A, A, 0,
+            1, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, [L] * 65, A, A, 0, 1, 0)
+
+
+def test_decode_validation(kvq):
+    L = _layer(kvq)
+    ok = dict(q=A, n_q_heads=24, T=1, n_kv=1024, chunk=256, scale=1 / 16, out_part=A,
+              lse_part=A, stream=0)
+
+    def call(**kw):
+        d = dict(ok)
+        d.update(kw)
+        kvq.kvq_decode_attn(L, **d)
+
+    def bad(status, **kw):
+        _raises(kvq, status, call, **kw)
+
+    bad(kvq.KVQ_ERR_INVALID_ARG, q=None)
+    bad(kvq.KVQ_ERR_ALIGNMENT, q=A + 2)
+    bad(kvq.KVQ_ERR_ALIGNMENT, out_part=A + 4)
+    bad(kvq.KVQ_ERR_INVALID_ARG, n_q_heads=25)
+    bad(kvq.KVQ_ERR_INVALID_ARG, T=0)
+    bad(kvq.KVQ_ERR_UNSUPPORTED, T=5)
+    bad(kvq.KVQ_ERR_UNSUPPORTED, n_q_heads=48, T=3)
+    bad(kvq.KVQ_ERR_INVALID_ARG, chunk=100)
+    bad(kvq.KVQ_ERR_INVALID_ARG, chunk=0)
+    bad(kvq.KVQ_ERR_INVALID_ARG, n_kv=1025)
+    bad(kvq.KVQ_ERR_INVALID_ARG, n_kv=3, T=4)
+    bad(kvq.KVQ_ERR_INVALID_ARG, scale=float("nan"))
+
+
+def test_merge_validation(kvq):
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_merge_lse, None, A, 4, 2, 256, A, A, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_merge_lse, A, A, 4, 0, 256, A, A, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_merge_lse, A, A, -1, 2, 256, A, A, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_merge_lse, A, A, 4, 2, 30, A, A, 0)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_merge_lse, A, A, 4, 2, 256, A + 4, A, 0)
+
+
+def test_prefill_validation(kvq):
+    L = _layer(kvq, capacity=4096)
+    ok = dict(q=A, n_q_heads=24, T=128, n_cached=1024, page=1024, scale=1 / 16, out=A, lse=A,
+              stream=0)
+
+    def call(**kw):
+        d = dict(ok)
+        d.update(kw)
+        kvq.kvq_prefill_attn(L, **d)
+
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, page=100)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, n_cached=4000)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, page_out=A)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, T=0)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, call, out=A + 4)
+
+
+def test_stream_validation(kvq):
+    L = _layer(kvq)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_stream_decode, [L], [L, _layer(kvq, head_dim=128)],
+            A, 24, 1, 1024, 256, 1 / 16, A, A, A, A, 0, 0)
+    with pytest.raises(ValueError):
+        kvq.kvq_stream_decode([L], [L], A, 24, 1, 1024, 256, 1 / 16, A, A, A, A, 0, 0)
+
+
+def test_workspace_query(kvq):
+    assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE, 16, 24, 4, 4, 256) == 0
+    assert kvq.kvq_workspace_bytes(99, 1, 1, 1, 1, 32) == ctypes.c_size_t(-1).value
