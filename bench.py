@@ -1,0 +1,420 @@
+"""Benchmark of the quantized-KV decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config verify262k|decode65k|stream262k|tiny]
+
+One step (default workload ``verify262k``: 16 attention layers, 24 query heads
+over 4 Q8_0/Q4_0 KV heads of 256, a 4-token speculative-verify batch against
+262,144 keys) is the whole decode hot path of one batch:
+
+  1. quantize-append the 4 new K/V rows of every layer (kvq_append, 1 launch),
+  2. split-KV GQA decode attention of all 16 layers, chunk 4,096
+     (kvq_decode_attn, 1 launch, per-chunk out + lse),
+  3. LSE merge of the 64 chunk partials of every row (kvq_merge_lse, 1 launch).
+
+``value`` is KV GB/s of the whole job: quantized KV bytes the step attends
+over (16 x 262,144 x 1,664 B = 6.98 GB) times steps, over the max-over-ranks
+device time.  Inputs are resident in HBM (the 7 GB cache is far larger than
+the 126 MB L2, so no flush is needed).  ``e2e`` is the same metric through the
+C-ABI with host buffers: every step copies q and the new rows from pinned host
+memory and copies out + lse back, inside the timed region.
+
+With --gpus N > 1 (torchrun, one rank per GPU, NCCL) every rank runs its own
+independent sequence (weak scaling, no data-path collective); ranks meet only
+at the timing barriers and the max-over-ranks reduction.
+
+``--impl reference`` times the CPU oracle (fp64, OpenMP) on a bounded sample of
+the same workload per step; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from quantized_kv_long_b200 import workload as wl  # noqa: E402
+
+METRIC = "q8_0/q4_0 decode attn: KV GB/s (% of HBM peak), query-tok/s at 262k ctx"
+FALLBACK_HBM_GBS = 6650.0
+KV_BYTES_PER_TOKEN_LAYER = lambda w: w.n_kv_heads * (w.head_dim // 32) * (34 + 18)  # noqa: E731
+
+
+# --------------------------------------------------------------------------- helpers
+
+def peaks() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max over ranks (identity when torch.distributed is not initialised)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None) -> None:
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                    rows.append(p)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+def gpu_id(torch, device) -> str:
+    """nvidia-smi -i argument for this device (its UUID when torch knows it)."""
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        return str(device.index)
+
+
+def source_hash(*names: str) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "quantized_kv_long_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel_files: tuple[str, ...]):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the kernel source as it is now (else None)."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        rec = json.load(open(p))
+    except Exception:
+        return None
+    if rec.get("source_hash") != source_hash(*kernel_files):
+        return None
+    return rec
+
+
+# --------------------------------------------------------------------------- our arm
+
+def fill_cache(kvq, torch, w: wl.Workload, device):
+    """Quantize the whole context of every layer into a device cache (setup,
+    untimed): rows [0, n_kv) drawn per layer by the seeded generator."""
+    cache = kvq.QuantizedKVCache(w.n_layers, w.n_kv_heads, w.head_dim, w.capacity, device=device)
+    for l in range(w.n_layers):
+        for start in range(0, w.n_kv, 131072):
+            stop = min(w.n_kv, start + 131072)
+            k = torch.from_numpy(wl.kv_rows(w, l, 0, start, stop)).to(device)
+            v = torch.from_numpy(wl.kv_rows(w, l, 1, start, stop)).to(device)
+            kvq.kvq_append(cache.layer(l), k, v, start, stop - start)
+    torch.cuda.synchronize(device)
+    return cache
+
+
+def run_ours(args, w: wl.Workload) -> dict | None:
+    import torch
+    import torch.distributed as dist
+    from quantized_kv_long_b200 import kvq
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+
+    L, T, Hq, D, n_kv, chunk = w.n_layers, w.T, w.n_q_heads, w.head_dim, w.n_kv, w.chunk
+    C = w.n_chunks
+    rows = L * T * Hq
+    cache = fill_cache(kvq, torch, w, device)
+    layers = cache.layers()
+    # the step's inputs: q and the T new rows of every layer (rows n_kv-T .. n_kv-1)
+    q_h = np.stack([wl.q_rows(w, l) for l in range(L)])
+    k_h = np.stack([wl.kv_rows(w, l, 0, n_kv - T, n_kv) for l in range(L)])
+    v_h = np.stack([wl.kv_rows(w, l, 1, n_kv - T, n_kv) for l in range(L)])
+    q = torch.from_numpy(q_h).to(device)
+    k_new = torch.from_numpy(k_h).to(device)
+    v_new = torch.from_numpy(v_h).to(device)
+    op = torch.empty((L, T, Hq, C, D), device=device)
+    lp = torch.empty((L, T, Hq, C), device=device)
+    out = torch.empty((L, T, Hq, D), device=device)
+    lse = torch.empty((L, T, Hq), device=device)
+
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+
+    def step(i=None):
+        kvq.kvq_append(layers, k_new, v_new, n_kv - T, T, stream)
+        if i is not None:
+            ev_dec[i][0].record(stream)
+        kvq.kvq_decode_attn(layers, q, Hq, T, n_kv, chunk, w.scale, op, lp, stream)
+        if i is not None:
+            ev_dec[i][1].record(stream)
+        kvq.kvq_merge_lse(op, lp, rows, C, D, out, lse, stream)
+
+    for _ in range(args.warmup):
+        step()
+    kvq.kvq_check(stream)
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id(torch, device)) as clocks:
+        barrier(device)
+        torch.cuda.synchronize(device)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+    kvq.kvq_check(stream)
+    ms_local = t0.elapsed_time(t1) / args.steps
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_dec)
+    ms = reduce_max(ms_local, device)
+    dec_ms_max = reduce_max(dec_ms, device)
+
+    # ---- e2e: the same step through the C ABI with host buffers
+    q_pin = torch.from_numpy(q_h).pin_memory()
+    k_pin = torch.from_numpy(k_h).pin_memory()
+    v_pin = torch.from_numpy(v_h).pin_memory()
+    out_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_pin = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(q_pin, non_blocking=True)
+        k_new.copy_(k_pin, non_blocking=True)
+        v_new.copy_(v_pin, non_blocking=True)
+        step()
+        out_pin.copy_(out, non_blocking=True)
+        lse_pin.copy_(lse, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, args.steps // 2)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, device)
+    h2d = q_pin.numel() * 2 + k_pin.numel() * 4 + v_pin.numel() * 4
+    d2h = out_pin.numel() * 4 + lse_pin.numel() * 4
+
+    # sanity: outputs are finite (the parity tests check them against the oracle)
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+
+    kv_bytes = L * n_kv * KV_BYTES_PER_TOKEN_LAYER(w)
+    peak, peak_kind = peaks()
+    cl = clocks.summary()
+    res = None
+    if rank == 0:
+        gbs = world * kv_bytes / (ms * 1e-3) / 1e9
+        achieved = kv_bytes / (dec_ms_max * 1e-3) / 1e9
+        tr = traffic_record(DECODE_SOURCES)
+        res = {
+            "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "q8_0 K / q4_0 V x f16 q, f32 accumulate", "data": "synthetic",
+            "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": w.n_kv_heads,
+                       "head_dim": D, "context": n_kv, "query_tokens": T, "chunk": chunk,
+                       "seed": w.seed, "kv_bytes_per_step": kv_bytes,
+                       "l2": "inputs larger than L2 (7 GB cache vs 126 MB)",
+                       "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
+            "query_tok_per_s": round(world * L * T / (ms * 1e-3), 1),
+            "pct_hbm_peak": round(100 * gbs / world / peak, 2),
+            "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 4)},
+            "roofline": {"bound": "hbm", "kernel": "kvq_decode_attn (16 layers, 1 launch)",
+                         "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": tr["dram_bytes_per_launch"] if tr else None,
+                         "launch_ms": round(dec_ms_max, 4)},
+            "gpu_launches": 3 * args.steps,
+            "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
+                       "reasons": cl["reasons"], "samples": cl["samples"]},
+        }
+    del cache
+    if world > 1:
+        dist.destroy_process_group()
+    return res
+
+
+DECODE_SOURCES = ("decode.cu", "ptx.cuh", "common.cuh")
+
+
+# --------------------------------------------------------------------------- oracle
+
+def oracle_sample(w: wl.Workload, layers: list[int], n_keys: int, threads_note: bool = True):
+    """Oracle decode of the given layers over their first n_keys keys (the
+    per-chunk partials plus the merge).  Returns (seconds, kv bytes)."""
+    import oracle
+    caches = []
+    for l in layers:
+        kc, vc = oracle.empty_cache(w.n_kv_heads, w.head_dim, w.capacity)
+        k = wl.kv_rows(w, l, 0, 0, n_keys)
+        v = wl.kv_rows(w, l, 1, 0, n_keys)
+        oracle.append(kc, vc, k, v, 0)
+        caches.append((kc, vc))
+    t = time.perf_counter()
+    for (kc, vc), l in zip(caches, layers):
+        p, pl = oracle.decode_attn(kc, vc, wl.q_rows(w, l), n_keys, w.chunk, w.scale)
+        oracle.merge_lse(p, pl)
+    dt = time.perf_counter() - t
+    return dt, len(layers) * n_keys * KV_BYTES_PER_TOKEN_LAYER(w)
+
+
+def cpu_baseline(w: wl.Workload, budget_s: float = 12.0) -> dict:
+    """The oracle as it stands, on this host's cores, over whole layers of the
+    workload until about budget_s of CPU time is spent."""
+    import oracle
+    tot_t, tot_b, done = 0.0, 0, []
+    for l in range(w.n_layers):
+        dt, b = oracle_sample(w, [l], w.n_kv)
+        tot_t += dt
+        tot_b += b
+        done.append(l)
+        if tot_t >= budget_s:
+            break
+    return {"value": round(tot_b / tot_t / 1e9, 3), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(done)} of {w.n_layers} layers, full {w.n_kv}-key context, "
+                      f"T={w.T}, {w.n_q_heads} q heads: fp64 decode partials + merge",
+            "seconds": round(tot_t, 2)}
+
+
+def run_reference(args, w: wl.Workload) -> dict | None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    # per step: one layer's first 16 chunks (65,536 keys), layers in turn
+    n_keys = min(w.n_kv, 16 * w.chunk)
+    for i in range(args.warmup):
+        oracle_sample(w, [i % w.n_layers], n_keys)
+    tot_t, tot_b = 0.0, 0
+    for i in range(args.steps):
+        dt, b = oracle_sample(w, [i % w.n_layers], n_keys)
+        tot_t += dt
+        tot_b += b
+    gbs = tot_b / tot_t / 1e9
+    ms = 1e3 * tot_t / args.steps
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 3), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "layers": w.n_layers, "q_heads": w.n_q_heads,
+                   "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "context": w.n_kv,
+                   "query_tokens": w.T, "chunk": w.chunk, "seed": w.seed},
+        "cpu_baseline": {"value": round(gbs, 3), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step one layer's first {n_keys} keys (all heads, "
+                                   f"T={w.T}): fp64 decode partials + merge"},
+        "e2e": {"value": round(gbs, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="verify262k", choices=["verify262k", "decode65k", "tiny"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = wl.WORKLOADS[args.config]
+    rank, world, _ = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, w)
+    else:
+        res = run_ours(args, w)
+        if res is not None and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(w)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -6,6 +6,8 @@
 // message for kvq_last_error().  Nothing here synchronises except kvq_check.
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <cmath>
 
@@ -167,6 +169,11 @@ kvq_status enqueue_decode(const kvq_layer *layers, int n_layers, const uint16_t 
     a.out_part = out_part;
     a.lse_part = lse_part;
     KVQ_TRY(status_word(&a.status));
+    // host-side test hooks (environment): the general kernel, a forced wait timeout
+    const char *ks = getenv("KVQ_DECODE_KERNEL");
+    a.force_simple = ks && strcmp(ks, "simple") == 0;
+    const char *tt = getenv("KVQ_TEST_DECODE_TIMEOUT");
+    a.test_timeout = tt && atoi(tt) != 0;
     if (!launch_decode(a, s))
         return set_error(KVQ_ERR_UNSUPPORTED, "kvq_decode_attn: no kernel for this shape");
     return check_launch("kvq_decode_attn");

@@ -67,6 +67,8 @@ struct DecodeArgs {
     const __half *q;
     float *out_part, *lse_part;
     unsigned int *status;  // device status word (bounded waits that ran out)
+    int force_simple;      // host test hook: use the general kernel
+    int test_timeout;      // host test hook: make the first wait run out
 };
 // Returns false (and launches nothing) if no kernel supports the shape.
 bool launch_decode(const DecodeArgs &a, cudaStream_t s);

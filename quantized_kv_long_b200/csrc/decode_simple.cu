@@ -146,9 +146,10 @@ bool launch_decode_simple(const DecodeArgs &a, cudaStream_t s)
     const size_t smem = decode_simple_smem(R, a.head_dim);
     if (smem > 227 * 1024)
         return false;
-    if (smem > 48 * 1024)
+    if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(decode_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+                             (int)smem) != cudaSuccess)
+        return false;
     const int n_chunks = (int)((a.n_kv + a.chunk - 1) / a.chunk);
     dim3 grid(n_chunks, a.n_kv_heads, a.n_layers);
     decode_simple_kernel<<<grid, SIMPLE_THREADS, smem, s>>>(a);

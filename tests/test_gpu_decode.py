@@ -23,6 +23,16 @@ def kvq():
     return m
 
 
+@pytest.fixture(params=["tc", "simple"])
+def kernel(request, monkeypatch):
+    """Run a case on the tiled tensor-core kernel and on the general kernel."""
+    if request.param == "simple":
+        monkeypatch.setenv("KVQ_DECODE_KERNEL", "simple")
+    else:
+        monkeypatch.delenv("KVQ_DECODE_KERNEL", raising=False)
+    return request.param
+
+
 def run_decode(kvq, cache, q, Hq, T, n_kv, chunk, scale, layers=None):
     n_layers = q.shape[0]
     D = q.shape[-1]
@@ -52,7 +62,7 @@ def check_case(kvq, w, n_layers, T, n_kv, chunk, cap=None):
         assert_attn_close(out[l], lse[l], mo, ml, f"merged layer {l}")
 
 
-def test_tiny_workload(kvq):
+def test_tiny_workload(kvq, kernel):
     """1 layer, 1 token, 1,024 context, seed 0: chunk 4,096 (one chunk) and 256."""
     w = wl.WORKLOADS["tiny"]
     check_case(kvq, w, 1, 1, 1024, 4096)
@@ -61,14 +71,14 @@ def test_tiny_workload(kvq):
 
 @pytest.mark.parametrize("T", [1, 2, 3, 4])
 @pytest.mark.parametrize("chunk", [256, 4096])
-def test_verify_batch_ragged_context(kvq, T, chunk):
+def test_verify_batch_ragged_context(kvq, T, chunk, kernel):
     """4,097 keys: a ragged last chunk; causal within the T new tokens."""
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=4097)
     check_case(kvq, w, 2, T, 4097, chunk)
 
 
 @pytest.mark.parametrize("T", [1, 4])
-def test_fully_masked_last_chunk(kvq, T):
+def test_fully_masked_last_chunk(kvq, T, kernel):
     """n_kv = 3*64 + 1: the last 64-key chunk holds one key, which only the
     last token sees; for the others that chunk must be (0, -inf)."""
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=193)
@@ -83,13 +93,13 @@ def test_other_shapes(kvq, D, H, Hq, T):
     check_case(kvq, w, 2, T, 700, 128)
 
 
-def test_minimal_context(kvq):
+def test_minimal_context(kvq, kernel):
     """n_kv == T: the first token sees exactly one key."""
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=4)
     check_case(kvq, w, 1, 4, 4, 64, cap=8)
 
 
-def test_sixteen_layers_one_call(kvq):
+def test_sixteen_layers_one_call(kvq, kernel):
     w = wl.small(wl.WORKLOADS["decode65k"], n_kv=2000)
     check_case(kvq, w, 16, 1, 2000, 512)
 
@@ -111,7 +121,7 @@ def test_merge_kernel_against_oracle(kvq):
     assert (out.cpu().numpy()[5] == 0).all() and lse.cpu().numpy()[5] == -np.inf
 
 
-def test_deterministic(kvq):
+def test_deterministic(kvq, kernel):
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=3000)
     cache, _ = fill_both(w, [0], 3000, 3000)
     q = q_all(w, [0], 4)
@@ -119,3 +129,34 @@ def test_deterministic(kvq):
     b = run_decode(kvq, cache, q, 24, 4, 3000, 1024, w.scale)
     for x, y in zip(a, b):
         assert np.array_equal(x, y)
+
+
+@pytest.mark.parametrize("n_kv,chunk", [(64, 64), (130, 64), (5000, 4096), (8192, 128)])
+def test_tc_stage_edges(kvq, n_kv, chunk):
+    """Chunks of one stage, a partial second stage (pairs without tokens),
+    chunks longer than the 4-stage ring, and many short chunks."""
+    w = wl.small(wl.WORKLOADS["verify262k"], n_kv=n_kv)
+    check_case(kvq, w, 1, 4, n_kv, chunk)
+    check_case(kvq, w, 1, 1, n_kv, chunk)
+
+
+def test_bounded_wait_times_out_and_context_survives(kvq, monkeypatch):
+    """A wait on a barrier that nothing completes runs out after about a
+    second: the kernel ends, kvq_check reports KVQ_ERR_TIMEOUT once, and the
+    next call on the same context is correct again."""
+    w = wl.small(wl.WORKLOADS["verify262k"], n_kv=512)
+    cache, orc = fill_both(w, [0], 512, 512)
+    q = q_all(w, [0], 4)
+    monkeypatch.setenv("KVQ_TEST_DECODE_TIMEOUT", "1")
+    qt = torch.from_numpy(q).cuda()
+    op = torch.empty((1, 4, 24, 1, 256), device="cuda")
+    lp = torch.empty((1, 4, 24, 1), device="cuda")
+    kvq.kvq_decode_attn(cache.layers(), qt, 24, 4, 512, 512, w.scale, op, lp)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_check()
+    assert e.value.status == kvq.KVQ_ERR_TIMEOUT
+    kvq.kvq_check()  # the status word was cleared
+    monkeypatch.delenv("KVQ_TEST_DECODE_TIMEOUT")
+    op2, lp2, out, lse = run_decode(kvq, cache, q, 24, 4, 512, 512, w.scale)
+    rp, rl = oracle.decode_attn(orc[0][0], orc[0][1], q[0], 512, 512, w.scale)
+    assert_attn_close(op2[0], lp2[0], rp, rl, "after timeout")
