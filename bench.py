@@ -400,10 +400,14 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="verify262k", choices=["verify262k", "decode65k", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="profile a smaller case of the same kernel: only this many layers")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = wl.WORKLOADS[args.config]
+    if args.layers is not None:
+        w = wl.small(w, n_layers=args.layers)
     rank, world, _ = dist_env()
     if args.impl == "reference":
         res = run_reference(args, w)

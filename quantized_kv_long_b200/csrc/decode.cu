@@ -11,24 +11,28 @@
 // lse = m + ln l.
 //
 // Layout of the work (head_dim 256, up to 24 rows = G*T):
-//  * one CTA per (layer, KV head, chunk) of 8 warps in four pairs; thread 0
-//    also issues the copies: a prologue of 4 stages, then each stage's slot
-//    is refilled as soon as all 8 warps have released it;
-//  * the chunk streams in stages of 64 tokens -- 64 K head-rows
-//    (17,408 B) and 64 V head-rows (9,216 B), each one contiguous 16-byte-
-//    aligned range in the head-major cache -- with cp.async.bulk into a ring
-//    of 4 shared-memory stages, completion tracked by mbarriers;
+//  * one CTA per (layer, KV head, chunk) of NPAIR warp pairs; thread 0 also
+//    issues the copies: a prologue of NS stages, then each stage's slot is
+//    refilled as soon as every warp has released it;
+//  * the chunk streams in stages of 16*NPAIR tokens -- that many K head-rows
+//    (272 B each) and V head-rows (144 B each), each one contiguous 16-byte-
+//    aligned range of the head-major cache -- with cp.async.bulk into a ring
+//    of NS shared-memory stages, completion tracked by mbarriers;
 //  * pair p owns tokens [16p, 16p+16) of every stage; warp 2p+hf of the pair
 //    owns head_dim half hf (Q8_0/Q4_0 blocks 4hf..4hf+3) of both contractions;
 //  * S^T = K Q^T on mma.sync m16n8k16 (rows = 16 tokens, columns = 8 query
-//    rows): int8 K is converted to f16 exactly, q is f16, each 32-element
-//    block's product is accumulated in fp32 and scaled by its fp32 d_b
-//    (times scale*log2 e), so only fp32 rounding separates S from the exact
-//    value.  The two halves' partial S are exchanged through shared memory;
-//  * online softmax per query row in base 2, with the running max shared by
-//    the 8 lanes of a column; a tile whose scores all stay below the running
-//    max skips the max reduction and the rescale (the max only needs to bound
-//    the scores for p <= 1; it is exact whenever it moves);
+//    rows).  The contraction index is permuted inside each 16-dim step so
+//    that a thread's four K bytes are contiguous (one 32-bit shared load for
+//    odd blocks, which start 4-byte aligned); Q's B-fragments live in shared
+//    memory in the same order.  int8 K converts to f16 exactly, q is f16, each
+//    32-element block's product is accumulated in fp32 and scaled by its fp32
+//    d_b (times scale*log2 e): only fp32 rounding separates S from exact.  The
+//    two halves' partial S are exchanged through shared memory;
+//  * online softmax per query row in base 2 with a lazy running max: it moves
+//    (exactly, with the rescale of O and l) only when a score exceeds it by
+//    more than TAU = 8, so p <= 2^8 -- harmless in fp32 and f16 -- and the
+//    cross-lane max and the rescale are almost never executed after the
+//    first tile.  The max then covers complete scores;
 //  * O^T += V^T P^T on mma.sync (rows = 16 head dims, columns = 8 query
 //    rows): Q4_0 nibbles become (u - 8) in f16 exactly; P is split into two
 //    f16 parts (P_hi + P_lo, ~2^-22 relative) that reach the B-operand layout
@@ -37,7 +41,7 @@
 //    each block costs two MMAs per tile but the PV side carries no fp16
 //    rounding of P: a single fp16 rounding of a dominant weight would cost
 //    up to |v^| * 2^-11, about 1.5e-2 on the x8 outlier channels;
-//  * at the end the four pairs' (m, l, O) merge through shared memory and the
+//  * at the end the pairs' (m, l, O) merge through shared memory and the
 //    chunk partial (out, lse) is written.
 // Every mbarrier wait is bounded (about one second of wall time); a wait that
 // runs out sets the device status word and the CTA falls through without
@@ -51,33 +55,36 @@ bool launch_decode_simple(const DecodeArgs &a, cudaStream_t s);
 
 namespace {
 
-constexpr int TOK = 64;                       // tokens per stage
+constexpr int NPAIR = 6;                      // warp pairs per CTA
+constexpr int WARPS = 2 * NPAIR;
+constexpr int THREADS = 32 * WARPS;
+constexpr int TOK = 16 * NPAIR;               // tokens per stage
 constexpr int NS = 4;                         // stages in the ring
 constexpr int KROW = 272, VROW = 144;         // head-row bytes at head_dim 256
-constexpr int STAGE_K = TOK * KROW;           // 17,408
-constexpr int STAGE_V = TOK * VROW;           // 9,216
+constexpr int STAGE_K = TOK * KROW;
+constexpr int STAGE_V = TOK * VROW;
 constexpr int STAGE_BYTES = STAGE_K + STAGE_V;
-constexpr int N_CONSUMER = 8;
-constexpr int THREADS = N_CONSUMER * 32;
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
+constexpr float TAU = 8.0f;                   // lazy-max slack (log2 units)
+constexpr float M_INIT = -1.0e30f;            // "no score yet", finite: ex2(s - M_INIT) stays defined
 
 template <int NT>
 struct __align__(16) DecodeSmem {
     uint8_t ring[NS][STAGE_BYTES];
-    float xs[4][2][2][NT * 4][32];  // partial S exchange [pair][parity][half][elem][lane]
-    float pm[4][32], pl[4][32];     // per-pair softmax stats per query row
+    float4 xs[NPAIR][2][2][NT][32];  // partial S exchange [pair][parity][half][n-tile][lane]
+    uint2 qf[2][8][NT][32];          // Q^T B-fragments [half][k-step][n-tile][lane]
+    float pm[NPAIR][32], pl[NPAIR][32];
     uint64_t full[NS], empty[NS], never;
     int abort;
 };
 
-// Two int8 (as a u16 pair: lo = 2 consecutive bytes, hi = 2 more) -> two half2
-// holding the exact integer values: (0x64 << 8 | (b ^ 0x80)) is 1024 + b + 128.
-__device__ __forceinline__ void s8x4_to_h2x2(uint32_t lo, uint32_t hi, uint32_t &h01,
-                                             uint32_t &h23)
+// Four int8 in a u32 -> two half2 holding the exact integers:
+// (0x64 << 8 | (b ^ 0x80)) is the f16 1152 + b.
+__device__ __forceinline__ void s8x4_to_h2x2(uint32_t w, uint32_t &h01, uint32_t &h23)
 {
-    const uint32_t w = ptx::prmt(lo, hi, 0x5410) ^ 0x80808080u;
+    w ^= 0x80808080u;
     const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
     h01 = ptx::h2_bits(__hsub2(ptx::bits_h2(ptx::prmt(w, 0x64646464u, 0x5140)), bias));
     h23 = ptx::h2_bits(__hsub2(ptx::bits_h2(ptx::prmt(w, 0x64646464u, 0x7362)), bias));
@@ -104,6 +111,20 @@ __device__ __forceinline__ uint32_t lds16(const uint8_t *p)
     return *reinterpret_cast<const uint16_t *>(p);
 }
 
+__device__ __forceinline__ uint32_t lds32(const uint8_t *p)
+{
+    return *reinterpret_cast<const uint32_t *>(p);
+}
+
+// The four K bytes [p, p+4) of a k-step; 4-byte aligned exactly when `aligned`
+// (a constant once the block loop is unrolled).
+__device__ __forceinline__ uint32_t k_word(const uint8_t *p, bool aligned)
+{
+    if (aligned)
+        return lds32(p);
+    return ptx::prmt(lds16(p), lds16(p + 2), 0x5410);
+}
+
 template <int NT>
 __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs a)
 {
@@ -126,24 +147,41 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             ptx::mbar_init(&sm.full[i], 1);
-            ptx::mbar_init(&sm.empty[i], N_CONSUMER);
+            ptx::mbar_init(&sm.empty[i], WARPS);
         }
         ptx::mbar_init(&sm.never, 1);
         sm.abort = 0;
         ptx::fence_mbar_init();
+    }
+    // Q^T B-fragments: entry (hf, ks, nt, lane) holds q[row nt*8 + lane/4] dims
+    // 128 hf + 16 ks + 4 (lane%4) .. +3 (the permuted k order; zero for padded rows)
+    {
+        const __half *qbase = a.q + (int64_t)layer * a.T * a.n_q_heads * 256;
+        for (int e = threadIdx.x; e < 2 * 8 * NT * 32; e += THREADS) {
+            const int ln = e & 31, nt = (e >> 5) % NT, ks = (e / (32 * NT)) & 7;
+            const int hf2 = e / (32 * NT * 8);
+            const int r = nt * 8 + (ln >> 2);
+            uint2 v = make_uint2(0u, 0u);
+            if (r < R) {
+                const int t = r / G, gq = r % G;
+                v = *reinterpret_cast<const uint2 *>(
+                    qbase + ((int64_t)t * a.n_q_heads + h * G + gq) * 256 + hf2 * 128 + ks * 16 +
+                    4 * (ln & 3));
+            }
+            sm.qf[hf2][ks][nt][ln] = v;
+        }
     }
     __syncthreads();
     volatile int *abort = &sm.abort;
 
     const int g = lane >> 2, cq = lane & 3;
     const int pair = warp >> 1, hf = warp & 1;
-    // accumulators of this warp: O^T for its 128 dims (8 m-tiles) x NT n-tiles
-    float o[8][NT][4];
+    float o[8][NT][4];  // O^T of this warp's 128 dims (8 m-tiles) x NT n-tiles
     float m2[NT][2], l2[NT][2];
 
     // ---------------------------------------------------------------- copies
-    // thread 0 issues stage s into slot s % NS once the slot's consumers released
-    // it (empty) and its previous copy landed (full); returns false on a timeout
+    // thread 0 issues stage st into slot st % NS once the slot's consumers
+    // released it (empty) and its previous copy landed (full); false on timeout
     auto issue = [&](int st) -> bool {
         const int slot = st % NS;
         const uint32_t round = st / NS;
@@ -163,283 +201,258 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs 
         for (; issued < NS && issued < n_stages; ++issued)
             issue(issued);
 
-    {
-        // ------------------------------------------------------------ consumers
-        // Q^T B-fragments for this warp's 8 k-steps (16 dims each) and NT n-tiles
-        uint32_t qf[8][NT][2];
-        const __half *qbase = a.q + (int64_t)layer * a.T * a.n_q_heads * 256;
+    const float dscale = a.scale * LOG2E;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int r = nt * 8 + g;
-            const bool live = r < R;
-            const int t = live ? r / G : 0, gq = live ? r % G : 0;
-            const uint32_t *qr = reinterpret_cast<const uint32_t *>(
-                qbase + ((int64_t)t * a.n_q_heads + h * G + gq) * 256 + hf * 128);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                qf[ks][nt][0] = live ? qr[(ks * 16 + 2 * cq) >> 1] : 0u;
-                qf[ks][nt][1] = live ? qr[(ks * 16 + 2 * cq + 8) >> 1] : 0u;
-            }
-        }
-        // key limit per owned column (query row): j <= n_kv - T + t; padded rows see nothing
-        // (relative to the chunk start c0; -1 sees nothing)
-        int lim[NT][2];
+    for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int r = nt * 8 + 2 * cq + k;
-                const int64_t l = a.n_kv - a.T + r / G - c0;
-                lim[nt][k] = r < R ? (int)(l < (int64_t)n_tok ? l : (int64_t)n_tok) : -1;
-            }
-        const float dscale = a.scale * LOG2E;
+            for (int i = 0; i < 4; ++i)
+                o[mt][nt][i] = 0.0f;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            m2[nt][k] = M_INIT;
+            l2[nt][k] = 0.0f;
+        }
+    if (a.test_timeout && lane == 0) {
+        // test hook: wait on a barrier that nothing completes
+        if (!ptx::mbar_wait_bounded(&sm.never, 0, abort, WAIT_LIMIT_NS)) {
+            *abort = 1;
+            report_timeout(a.status);
+        }
+    }
+    __syncwarp();
+
+    int par = 0;
+    bool aborted = false;
+    for (int s = 0; s < n_stages; ++s) {
+        const int slot = s % NS;
+        if (!aborted) {
+            bool ok = true;
+            if (lane == 0)
+                ok = ptx::mbar_wait_bounded(&sm.full[slot], (s / NS) & 1, abort, WAIT_LIMIT_NS);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                if (lane == 0 && !*abort) {
+                    *abort = 1;
+                    report_timeout(a.status);
+                }
+                aborted = true;
+            }
+        }
+        const int valid = min(16, n_tok - s * TOK - 16 * pair);  // tokens of this pair's tile
+        // both warps of a pair see the same `valid`, so both take the exchange barrier
+        if (valid > 0) {
+            const uint8_t *ks = sm.ring[slot] + (16 * pair) * KROW;
+            const uint8_t *vs = sm.ring[slot] + STAGE_K + (16 * pair) * VROW;
+            const int j0 = s * TOK + 16 * pair;  // key of token 0, relative to c0
+            float sacc[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    o[mt][nt][i] = 0.0f;
+                    sacc[nt][i] = 0.0f;
+            if (!aborted) {
+                // ---- S^T partial over this warp's 4 blocks, exact per-block scale
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+                for (int bb = 0; bb < 4; ++bb) {
+                    const int b = 4 * hf + bb;  // parity of b is the parity of bb
+                    const uint8_t *r0 = ks + g * KROW + 34 * b;
+                    const uint8_t *r1 = r0 + 8 * KROW;
+                    const float dk0 = __half2float(__ushort_as_half((unsigned short)lds16(r0))) * dscale;
+                    const float dk1 = __half2float(__ushort_as_half((unsigned short)lds16(r1))) * dscale;
+                    float blk[NT][4];
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                m2[nt][k] = -INFINITY;
-                l2[nt][k] = 0.0f;
-            }
-        if (a.test_timeout && lane == 0) {
-            // test hook: wait on a barrier that nothing completes
-            if (!ptx::mbar_wait_bounded(&sm.never, 0, abort, WAIT_LIMIT_NS)) {
-                *abort = 1;
-                report_timeout(a.status);
-            }
-        }
-        __syncwarp();
-
-        int par = 0;
-        for (int s = 0; s < n_stages; ++s) {
-            const int slot = s % NS;
-            bool ok = true;
-            if (lane == 0)
-                ok = ptx::mbar_wait_bounded(&sm.full[slot], (s / NS) & 1, abort, WAIT_LIMIT_NS);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok && lane == 0 && !*abort) {
-                *abort = 1;
-                report_timeout(a.status);
-            }
-            const int valid = min(16, n_tok - s * TOK - 16 * pair);  // tokens of this pair's tile
-            const bool aborted = __shfl_sync(0xffffffffu, lane == 0 ? *abort : 0, 0) != 0;
-            const bool run = valid > 0 && !aborted;
-            // both warps of a pair see the same `valid`; `abort` may differ, so the exchange
-            // barrier below is taken whenever valid > 0
-            if (valid > 0) {
-                const uint8_t *ks = sm.ring[slot] + (16 * pair) * KROW;
-                const uint8_t *vs = sm.ring[slot] + STAGE_K + (16 * pair) * VROW;
-                const int j0 = s * TOK + 16 * pair;  // key of token 0, relative to c0
-                float sacc[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        sacc[nt][i] = 0.0f;
-                if (run) {
-                    // ---- S^T partial over this warp's 4 blocks, exact per-block scale
-#pragma unroll
-                    for (int bb = 0; bb < 4; ++bb) {
-                        const int b = 4 * hf + bb;
-                        const uint8_t *r0 = ks + g * KROW + 34 * b;
-                        const uint8_t *r1 = r0 + 8 * KROW;
-                        const float dk0 = __half2float(__ushort_as_half((unsigned short)lds16(r0))) * dscale;
-                        const float dk1 = __half2float(__ushort_as_half((unsigned short)lds16(r1))) * dscale;
-                        float blk[NT][4];
-#pragma unroll
-                        for (int s2 = 0; s2 < 2; ++s2) {
-                            const int off = 2 + 16 * s2 + 2 * cq;
-                            uint32_t af[4];
-                            s8x4_to_h2x2(lds16(r0 + off), lds16(r0 + off + 8), af[0], af[2]);
-                            s8x4_to_h2x2(lds16(r1 + off), lds16(r1 + off + 8), af[1], af[3]);
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                if (s2 == 0) {
-                                    const float z[4] = {0.f, 0.f, 0.f, 0.f};
-                                    ptx::mma_f16_16816(blk[nt], af, qf[2 * bb][nt][0],
-                                                       qf[2 * bb][nt][1], z);
-                                } else {
-                                    ptx::mma_f16_16816(blk[nt], af, qf[2 * bb + 1][nt][0],
-                                                       qf[2 * bb + 1][nt][1], blk[nt]);
-                                }
-                            }
-                        }
+                    for (int s2 = 0; s2 < 2; ++s2) {
+                        const int off = 2 + 16 * s2 + 4 * cq;
+                        uint32_t af[4];
+                        s8x4_to_h2x2(k_word(r0 + off, (bb & 1) != 0), af[0], af[2]);
+                        s8x4_to_h2x2(k_word(r1 + off, (bb & 1) != 0), af[1], af[3]);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            sacc[nt][0] = fmaf(dk0, blk[nt][0], sacc[nt][0]);
-                            sacc[nt][1] = fmaf(dk0, blk[nt][1], sacc[nt][1]);
-                            sacc[nt][2] = fmaf(dk1, blk[nt][2], sacc[nt][2]);
-                            sacc[nt][3] = fmaf(dk1, blk[nt][3], sacc[nt][3]);
+                            const uint2 qb = sm.qf[hf][2 * bb + s2][nt][lane];
+                            if (s2 == 0) {
+                                const float z[4] = {0.f, 0.f, 0.f, 0.f};
+                                ptx::mma_f16_16816(blk[nt], af, qb.x, qb.y, z);
+                            } else {
+                                ptx::mma_f16_16816(blk[nt], af, qb.x, qb.y, blk[nt]);
+                            }
                         }
                     }
-                }
-                // ---- exchange partial S with the other half of the pair
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        sm.xs[pair][par][hf][nt * 4 + i][lane] = sacc[nt][i];
-                ptx::named_bar_sync(1 + pair, 64);
-                float sv[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        sv[nt][i] = sacc[nt][i] + sm.xs[pair][par][hf ^ 1][nt * 4 + i][lane];
-                par ^= 1;
-
-                if (run) {
-                    // ---- mask (ragged tail of the chunk, causal rows of the verify batch)
-                    const bool need_mask = valid < 16 || c0 + j0 + 15 > a.n_kv - a.T;
-                    if (need_mask) {
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int tt = g + 8 * (i >> 1);
-                                if (tt >= valid || j0 + tt > lim[nt][i & 1])
-                                    sv[nt][i] = -INFINITY;
-                            }
+                    for (int nt = 0; nt < NT; ++nt) {
+                        sacc[nt][0] = fmaf(dk0, blk[nt][0], sacc[nt][0]);
+                        sacc[nt][1] = fmaf(dk0, blk[nt][1], sacc[nt][1]);
+                        sacc[nt][2] = fmaf(dk1, blk[nt][2], sacc[nt][2]);
+                        sacc[nt][3] = fmaf(dk1, blk[nt][3], sacc[nt][3]);
                     }
-                    // ---- online softmax (base 2)
-                    float tmax[NT][2];
-                    bool up = false;
+                }
+            }
+            // ---- exchange partial S with the other half of the pair
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                sm.xs[pair][par][hf][nt][lane] =
+                    make_float4(sacc[nt][0], sacc[nt][1], sacc[nt][2], sacc[nt][3]);
+            ptx::named_bar_sync(1 + pair, 64);
+            float sv[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float4 x = sm.xs[pair][par][hf ^ 1][nt][lane];
+                sv[nt][0] = sacc[nt][0] + x.x;
+                sv[nt][1] = sacc[nt][1] + x.y;
+                sv[nt][2] = sacc[nt][2] + x.z;
+                sv[nt][3] = sacc[nt][3] + x.w;
+            }
+            par ^= 1;
+
+            if (!aborted) {
+                // ---- mask (ragged tail of the chunk, causal rows of the verify batch,
+                //      padded rows)
+                const bool need_mask = valid < 16 || c0 + j0 + 15 > a.n_kv - a.T;
+                if (need_mask) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int tt = g + 8 * (i >> 1);
+                            const int r = nt * 8 + 2 * cq + (i & 1);
+                            const bool vis = tt < valid && r < R &&
+                                             c0 + j0 + tt <= a.n_kv - a.T + r / G;
+                            if (!vis)
+                                sv[nt][i] = -INFINITY;
+                        }
+                }
+                // ---- online softmax (base 2), lazy running max
+                float tmax[NT][2];
+                bool up = false;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        tmax[nt][k] = fmaxf(sv[nt][k], sv[nt][2 + k]);
+                        up |= tmax[nt][k] > m2[nt][k] + TAU;
+                    }
+                if (__any_sync(0xffffffffu, up)) {
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int k = 0; k < 2; ++k) {
-                            tmax[nt][k] = fmaxf(sv[nt][k], sv[nt][2 + k]);
-                            up |= tmax[nt][k] > m2[nt][k];
-                        }
-                    if (__any_sync(0xffffffffu, up)) {
+                            float v = tmax[nt][k];
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                            const float mn = fmaxf(m2[nt][k], v);
+                            const float al = ptx::ex2(m2[nt][k] - mn);
+                            m2[nt][k] = mn;
+                            l2[nt][k] *= al;
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                            for (int k = 0; k < 2; ++k) {
-                                float v = tmax[nt][k];
-                                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                                const float mn = fmaxf(m2[nt][k], v);
-                                const float al = (mn == -INFINITY) ? 1.0f : ptx::ex2(m2[nt][k] - mn);
-                                m2[nt][k] = mn;
-                                l2[nt][k] *= al;
-#pragma unroll
-                                for (int mt = 0; mt < 8; ++mt) {
-                                    o[mt][nt][k] *= al;
-                                    o[mt][nt][2 + k] *= al;
-                                }
+                            for (int mt = 0; mt < 8; ++mt) {
+                                o[mt][nt][k] *= al;
+                                o[mt][nt][2 + k] *= al;
                             }
+                        }
+                }
+                // P = P_hi + P_lo (two f16 parts, residual ~2^-22 relative), moved to the
+                // B-operand layout (tokens along k) with movmatrix.trans
+                uint32_t ph[NT][2], pl[NT][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float p[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        p[i] = ptx::ex2(sv[nt][i] - m2[nt][i & 1]);
+                    l2[nt][0] += p[0] + p[2];
+                    l2[nt][1] += p[1] + p[3];
+                    const __half2 h01 = __floats2half2_rn(p[0], p[1]);
+                    const __half2 h23 = __floats2half2_rn(p[2], p[3]);
+                    const __half2 r01 = __floats2half2_rn(p[0] - __low2float(h01),
+                                                          p[1] - __high2float(h01));
+                    const __half2 r23 = __floats2half2_rn(p[2] - __low2float(h23),
+                                                          p[3] - __high2float(h23));
+                    ph[nt][0] = ptx::movmatrix_trans(ptx::h2_bits(h01));
+                    ph[nt][1] = ptx::movmatrix_trans(ptx::h2_bits(h23));
+                    pl[nt][0] = ptx::movmatrix_trans(ptx::h2_bits(r01));
+                    pl[nt][1] = ptx::movmatrix_trans(ptx::h2_bits(r23));
+                }
+                // ---- O^T += V^T (P d_v)^T over this warp's 4 blocks
+                const uint8_t *v0 = vs + (2 * cq) * VROW;  // tokens 2c, 2c+1, 2c+8, 2c+9
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    const int b = 4 * hf + bb;
+                    const uint8_t *vb = v0 + 18 * b;
+                    uint32_t d0 = lds16(vb), d1 = lds16(vb + VROW);
+                    uint32_t d2 = lds16(vb + 8 * VROW), d3 = lds16(vb + 9 * VROW);
+                    if (valid < 16) {  // tokens past the chunk end may hold stale bytes
+                        if (2 * cq >= valid) d0 = 0;
+                        if (2 * cq + 1 >= valid) d1 = 0;
+                        if (2 * cq + 8 >= valid) d2 = 0;
+                        if (2 * cq + 9 >= valid) d3 = 0;
                     }
-                    // P = P_hi + P_lo (two f16 parts, residual ~2^-22 relative), moved to the
-                    // B-operand layout (tokens along k) with movmatrix.trans
-                    uint32_t ph[NT][2], pl[NT][2];
+                    const __half2 dA = ptx::bits_h2(ptx::prmt(d0, d1, 0x5410));
+                    const __half2 dB = ptx::bits_h2(ptx::prmt(d2, d3, 0x5410));
+                    const uint32_t x0 = lds16(vb + 2 + 2 * g), x1 = lds16(vb + VROW + 2 + 2 * g);
+                    const uint32_t x2 = lds16(vb + 8 * VROW + 2 + 2 * g);
+                    const uint32_t x3 = lds16(vb + 9 * VROW + 2 + 2 * g);
+                    const uint32_t wA0 = ptx::prmt(x0, x1, 0x0400);  // byte 2g of tokens 2c, 2c+1
+                    const uint32_t wA1 = ptx::prmt(x0, x1, 0x0501);  // byte 2g+1
+                    const uint32_t wB0 = ptx::prmt(x2, x3, 0x0400);  // tokens 2c+8, 2c+9
+                    const uint32_t wB1 = ptx::prmt(x2, x3, 0x0501);
+                    const uint32_t alo[4] = {nib_lo(wA0), nib_lo(wA1), nib_lo(wB0), nib_lo(wB1)};
+                    const uint32_t ahi[4] = {nib_hi(wA0), nib_hi(wA1), nib_hi(wB0), nib_hi(wB1)};
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        float p[4];
+                        // P d_v as hi + lo without loss: hi = RN(P_hi d), the exact
+                        // product error fma(P_hi, d, -hi), plus P_lo d
+                        uint32_t bh[2], bl[2];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float mm = m2[nt][i & 1];
-                            p[i] = (mm == -INFINITY) ? 0.0f : ptx::ex2(sv[nt][i] - mm);
+                        for (int k = 0; k < 2; ++k) {
+                            const __half2 d = k == 0 ? dA : dB;
+                            const __half2 a_hi = ptx::bits_h2(ph[nt][k]);
+                            const __half2 hi = __hmul2_rn(a_hi, d);
+                            const __half2 err = __hfma2(a_hi, d, __hneg2(hi));
+                            bh[k] = ptx::h2_bits(hi);
+                            bl[k] = ptx::h2_bits(__hfma2(ptx::bits_h2(pl[nt][k]), d, err));
                         }
-                        l2[nt][0] += p[0] + p[2];
-                        l2[nt][1] += p[1] + p[3];
-                        const __half2 h01 = __floats2half2_rn(p[0], p[1]);
-                        const __half2 h23 = __floats2half2_rn(p[2], p[3]);
-                        const __half2 r01 = __floats2half2_rn(p[0] - __low2float(h01),
-                                                              p[1] - __high2float(h01));
-                        const __half2 r23 = __floats2half2_rn(p[2] - __low2float(h23),
-                                                              p[3] - __high2float(h23));
-                        ph[nt][0] = ptx::movmatrix_trans(ptx::h2_bits(h01));
-                        ph[nt][1] = ptx::movmatrix_trans(ptx::h2_bits(h23));
-                        pl[nt][0] = ptx::movmatrix_trans(ptx::h2_bits(r01));
-                        pl[nt][1] = ptx::movmatrix_trans(ptx::h2_bits(r23));
+                        ptx::mma_f16_16816(o[2 * bb][nt], alo, bh[0], bh[1], o[2 * bb][nt]);
+                        ptx::mma_f16_16816(o[2 * bb][nt], alo, bl[0], bl[1], o[2 * bb][nt]);
+                        ptx::mma_f16_16816(o[2 * bb + 1][nt], ahi, bh[0], bh[1], o[2 * bb + 1][nt]);
+                        ptx::mma_f16_16816(o[2 * bb + 1][nt], ahi, bl[0], bl[1], o[2 * bb + 1][nt]);
                     }
-                    // ---- O^T += V^T (P d_v)^T over this warp's 4 blocks
-                    const uint8_t *v0 = vs + (2 * cq) * VROW;  // tokens 2c, 2c+1, 2c+8, 2c+9
-#pragma unroll
-                    for (int bb = 0; bb < 4; ++bb) {
-                        const int b = 4 * hf + bb;
-                        const uint8_t *vb = v0 + 18 * b;
-                        uint32_t d0 = lds16(vb), d1 = lds16(vb + VROW);
-                        uint32_t d2 = lds16(vb + 8 * VROW), d3 = lds16(vb + 9 * VROW);
-                        if (need_mask) {  // tokens past the chunk end may hold stale bytes
-                            if (2 * cq >= valid) d0 = 0;
-                            if (2 * cq + 1 >= valid) d1 = 0;
-                            if (2 * cq + 8 >= valid) d2 = 0;
-                            if (2 * cq + 9 >= valid) d3 = 0;
-                        }
-                        const __half2 dA = ptx::bits_h2(d0 | (d1 << 16));
-                        const __half2 dB = ptx::bits_h2(d2 | (d3 << 16));
-                        const uint32_t x0 = lds16(vb + 2 + 2 * g), x1 = lds16(vb + VROW + 2 + 2 * g);
-                        const uint32_t x2 = lds16(vb + 8 * VROW + 2 + 2 * g);
-                        const uint32_t x3 = lds16(vb + 9 * VROW + 2 + 2 * g);
-                        const uint32_t wA0 = ptx::prmt(x0, x1, 0x0400);  // byte 2g of tokens 2c, 2c+1
-                        const uint32_t wA1 = ptx::prmt(x0, x1, 0x0501);  // byte 2g+1
-                        const uint32_t wB0 = ptx::prmt(x2, x3, 0x0400);  // tokens 2c+8, 2c+9
-                        const uint32_t wB1 = ptx::prmt(x2, x3, 0x0501);
-                        const uint32_t alo[4] = {nib_lo(wA0), nib_lo(wA1), nib_lo(wB0), nib_lo(wB1)};
-                        const uint32_t ahi[4] = {nib_hi(wA0), nib_hi(wA1), nib_hi(wB0), nib_hi(wB1)};
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            // P d_v as hi + lo without loss: hi = RN(P_hi d), the exact
-                            // product error fma(P_hi, d, -hi), plus P_lo d
-                            uint32_t bh[2], bl[2];
-#pragma unroll
-                            for (int k = 0; k < 2; ++k) {
-                                const __half2 d = k == 0 ? dA : dB;
-                                const __half2 a_hi = ptx::bits_h2(ph[nt][k]);
-                                const __half2 hi = __hmul2_rn(a_hi, d);
-                                const __half2 err = __hfma2(a_hi, d, __hneg2(hi));
-                                bh[k] = ptx::h2_bits(hi);
-                                bl[k] = ptx::h2_bits(__hfma2(ptx::bits_h2(pl[nt][k]), d, err));
-                            }
-                            ptx::mma_f16_16816(o[2 * bb][nt], alo, bh[0], bh[1], o[2 * bb][nt]);
-                            ptx::mma_f16_16816(o[2 * bb][nt], alo, bl[0], bl[1], o[2 * bb][nt]);
-                            ptx::mma_f16_16816(o[2 * bb + 1][nt], ahi, bh[0], bh[1], o[2 * bb + 1][nt]);
-                            ptx::mma_f16_16816(o[2 * bb + 1][nt], ahi, bl[0], bl[1], o[2 * bb + 1][nt]);
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0)
-                ptx::mbar_arrive(&sm.empty[slot]);
-            if (threadIdx.x == 0 && issued < n_stages && !*abort) {
-                if (issue(issued)) {
-                    ++issued;
-                } else if (!*abort) {
-                    *abort = 1;
-                    report_timeout(a.status);
                 }
             }
         }
-        // per-row sums over the 8 lanes that share a column
+        __syncwarp();
+        if (lane == 0)
+            ptx::mbar_arrive(&sm.empty[slot]);
+        if (threadIdx.x == 0 && issued < n_stages && !*abort) {
+            if (issue(issued)) {
+                ++issued;
+            } else if (!*abort) {
+                *abort = 1;
+                report_timeout(a.status);
+            }
+        }
+    }
+    // per-row sums over the 8 lanes that share a column
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            float v = l2[nt][k];
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 16);
+            l2[nt][k] = v;
+        }
+    if (hf == 0 && g == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
-                float v = l2[nt][k];
-                v += __shfl_xor_sync(0xffffffffu, v, 4);
-                v += __shfl_xor_sync(0xffffffffu, v, 8);
-                v += __shfl_xor_sync(0xffffffffu, v, 16);
-                l2[nt][k] = v;
+                sm.pm[pair][nt * 8 + 2 * cq + k] = m2[nt][k];
+                sm.pl[pair][nt * 8 + 2 * cq + k] = l2[nt][k];
             }
-        if (hf == 0 && g == 0) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    sm.pm[pair][nt * 8 + 2 * cq + k] = m2[nt][k];
-                    sm.pl[pair][nt * 8 + 2 * cq + k] = l2[nt][k];
-                }
-        }
     }
     if (threadIdx.x == 0) {
         // drain: every issued copy has landed before the ring is reused or freed
@@ -454,50 +467,50 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs 
 
     // ---------------------------------------------------------------- merge pairs
     constexpr int NCOL = NT * 8;
-    float *obuf = reinterpret_cast<float *>(sm.ring);  // [4][NCOL][256]
-    {
+    static_assert(sizeof(float) * NPAIR * NCOL * 256 <= sizeof(uint8_t) * NS * STAGE_BYTES,
+                  "merge buffer must fit in the ring");
+    float *obuf = reinterpret_cast<float *>(sm.ring);  // [NPAIR][NCOL][256]
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int col = nt * 8 + 2 * cq + k;
-                float M = -INFINITY;
+        for (int k = 0; k < 2; ++k) {
+            const int col = nt * 8 + 2 * cq + k;
+            float M = M_INIT;
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    M = fmaxf(M, sm.pm[p][col]);
-                float L = 0.0f;
+            for (int p = 0; p < NPAIR; ++p)
+                M = fmaxf(M, sm.pm[p][col]);
+            float L = 0.0f;
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    if (sm.pm[p][col] != -INFINITY)
-                        L += sm.pl[p][col] * ptx::ex2(sm.pm[p][col] - M);
-                const float f = (L > 0.0f && m2[nt][k] != -INFINITY) ? ptx::ex2(m2[nt][k] - M) / L : 0.0f;
+            for (int p = 0; p < NPAIR; ++p)
+                L += sm.pl[p][col] * ptx::ex2(sm.pm[p][col] - M);
+            const float f = (L > 0.0f) ? ptx::ex2(m2[nt][k] - M) / L : 0.0f;
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                    const int b = 4 * hf + (mt >> 1);
-                    const int dbase = 32 * b + ((mt & 1) ? 16 : 0) + 2 * g;
-                    obuf[(pair * NCOL + col) * 256 + dbase] = o[mt][nt][k] * f;
-                    obuf[(pair * NCOL + col) * 256 + dbase + 1] = o[mt][nt][2 + k] * f;
-                }
+            for (int mt = 0; mt < 8; ++mt) {
+                const int b = 4 * hf + (mt >> 1);
+                const int dbase = 32 * b + ((mt & 1) ? 16 : 0) + 2 * g;
+                obuf[(pair * NCOL + col) * 256 + dbase] = o[mt][nt][k] * f;
+                obuf[(pair * NCOL + col) * 256 + dbase + 1] = o[mt][nt][2 + k] * f;
             }
-    }
+        }
     __syncthreads();
     const int Hq = a.n_q_heads;
     for (int idx = threadIdx.x; idx < R * 256; idx += THREADS) {
         const int col = idx >> 8, dim = idx & 255;
-        const float v = obuf[(0 * NCOL + col) * 256 + dim] + obuf[(1 * NCOL + col) * 256 + dim] +
-                        obuf[(2 * NCOL + col) * 256 + dim] + obuf[(3 * NCOL + col) * 256 + dim];
+        float v = 0.0f;
+#pragma unroll
+        for (int p = 0; p < NPAIR; ++p)
+            v += obuf[(p * NCOL + col) * 256 + dim];
         const int t = col / G, gq = col % G;
         const int64_t row = ((int64_t)layer * a.T + t) * Hq + h * G + gq;
         a.out_part[(row * C + c) * 256 + dim] = v;
     }
     for (int col = threadIdx.x; col < R; col += THREADS) {
-        float M = -INFINITY;
-        for (int p = 0; p < 4; ++p)
+        float M = M_INIT;
+        for (int p = 0; p < NPAIR; ++p)
             M = fmaxf(M, sm.pm[p][col]);
         float L = 0.0f;
-        for (int p = 0; p < 4; ++p)
-            if (sm.pm[p][col] != -INFINITY)
-                L += sm.pl[p][col] * ptx::ex2(sm.pm[p][col] - M);
+        for (int p = 0; p < NPAIR; ++p)
+            L += sm.pl[p][col] * ptx::ex2(sm.pm[p][col] - M);
         const int t = col / G, gq = col % G;
         const int64_t row = ((int64_t)layer * a.T + t) * Hq + h * G + gq;
         a.lse_part[row * C + c] = (L > 0.0f) ? (M + log2f(L)) * LN2 : -INFINITY;
