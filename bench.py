@@ -317,6 +317,101 @@ def run_ours(args, w: wl.Workload) -> dict | None:
 
 
 DECODE_SOURCES = ("decode.cu", "ptx.cuh", "common.cuh")
+PREFILL_METRIC = "q8_0/q4_0 chunked prefill attn: TFLOP/s (% of tensor peak), query-tok/s at 262k ctx"
+
+
+def prefill_flops(w: wl.Workload) -> float:
+    """QK^T and PV multiply-adds of every visible (query row, key) pair, x2 flop."""
+    visible = sum(w.n_cached + t + 1 for t in range(w.T))
+    return 2.0 * 2.0 * w.head_dim * w.n_q_heads * visible * w.n_layers
+
+
+def tensor_peak() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (bf16 sustained)"
+    except Exception:
+        return 1400.0, "fallback (sustained)"
+
+
+def run_prefill(args, w: wl.Workload) -> dict | None:
+    """The prefill262k step: append the 2,048 new rows of every layer, then
+    prefill attention of all 16 layers (one launch each)."""
+    import torch
+    import torch.distributed as dist
+    from quantized_kv_long_b200 import kvq
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    L, T, Hq, D, nc = w.n_layers, w.T, w.n_q_heads, w.head_dim, w.n_cached
+    cache = fill_cache(kvq, torch, wl.small(w, n_kv=nc + T), device)
+    layers = cache.layers()
+    q = torch.from_numpy(np.stack([wl.q_rows(w, l) for l in range(L)])).to(device)
+    k_new = torch.from_numpy(np.stack([wl.kv_rows(w, l, 0, nc, nc + T) for l in range(L)])).to(device)
+    v_new = torch.from_numpy(np.stack([wl.kv_rows(w, l, 1, nc, nc + T) for l in range(L)])).to(device)
+    out = torch.empty((L, T, Hq, D), device=device)
+    lse = torch.empty((L, T, Hq), device=device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+
+    def step(i=None):
+        kvq.kvq_append(layers, k_new, v_new, nc, T, stream)
+        if i is not None:
+            ev[i][0].record(stream)
+        kvq.kvq_prefill_attn(layers, q, Hq, T, nc, w.page, w.scale, out, lse, stream=stream)
+        if i is not None:
+            ev[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    kvq.kvq_check(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id(torch, device)) as clocks:
+        barrier(device)
+        torch.cuda.synchronize(device)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+    kvq.kvq_check(stream)
+    ms = reduce_max(t0.elapsed_time(t1) / args.steps, device)
+    k_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev), device)
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    fl = prefill_flops(w)
+    peak, kind = tensor_peak()
+    cl = clocks.summary()
+    res = None
+    if rank == 0:
+        res = {
+            "metric": PREFILL_METRIC, "value": round(world * fl / (ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16 (K, V, P dequantized on chip), f32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": w.n_kv_heads,
+                       "head_dim": D, "cached": nc, "new_tokens": T, "seed": w.seed,
+                       "flop_per_step": fl},
+            "query_tok_per_s": round(world * L * T / (ms * 1e-3), 1),
+            "roofline": {"bound": "tensor", "kernel": "kvq_prefill_attn (16 layers, 1 launch)",
+                         "achieved": round(fl / (k_ms * 1e-3) / 1e12, 2), "peak": peak,
+                         "peak_kind": kind, "unit": "TFLOP/s",
+                         "frac": round(fl / (k_ms * 1e-3) / 1e12 / peak, 4), "traffic": None,
+                         "launch_ms": round(k_ms, 3)},
+            "gpu_launches": 2 * args.steps,
+            "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
+                       "reasons": cl["reasons"], "samples": cl["samples"]},
+        }
+    del cache
+    if world > 1:
+        dist.destroy_process_group()
+    return res
 
 
 # --------------------------------------------------------------------------- oracle
@@ -398,7 +493,8 @@ def main(argv=None) -> int:
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="verify262k", choices=["verify262k", "decode65k", "tiny"])
+    ap.add_argument("--config", default="verify262k",
+                    choices=["verify262k", "decode65k", "tiny", "prefill262k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="profile a smaller case of the same kernel: only this many layers")
@@ -411,6 +507,8 @@ def main(argv=None) -> int:
     rank, world, _ = dist_env()
     if args.impl == "reference":
         res = run_reference(args, w)
+    elif w.mode == "prefill":
+        res = run_prefill(args, w)
     else:
         res = run_ours(args, w)
         if res is not None and world == 1 and not args.no_cpu_baseline:

@@ -192,23 +192,29 @@ kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t r
 
 /* Prefill attention of T new query tokens per layer over n_cached + T keys
  * (the T new rows must already be appended at rows [n_cached, n_cached+T));
- * token t sees keys j <= n_cached + t.  Keys are processed page by page
- * (`page` keys each) with an online LSE merge across pages; K and V tiles are
- * dequantized on chip and the two contractions run on the tensor cores with
- * fp32 accumulation.
+ * token t sees keys j <= n_cached + t.  Keys are processed in tiles with an
+ * online LSE merge carried across pages of keys inside the kernel.  Rows that
+ * see at least 16,384 keys run on the tensor cores (tcgen05): K tiles are
+ * dequantized on chip to an exact two-part f16 sum (so the logits carry only
+ * fp32 rounding), V tiles and P to f16 (one rounding each), fp32
+ * accumulation in tensor memory; the V and P rounding errors average over the
+ * visible keys (measured max-abs error 2.2e-4 at 16,384 keys and 8.8e-5 at
+ * 262,144 on N(0,1) K/V with x8 outlier channels).  Rows that see fewer keys
+ * run an exact fp32 kernel on the CUDA cores.
+ * The tensor-core path needs head_dim 256; other head_dims take the exact
+ * kernel.
  * Source: "Online Log-Sum-Exp prefill & pipelined prefetch" of the RX 9070 XT
  * page (chunked prefill over streamed pages with online LSE accumulation).
  *  q         device fp16 bits [n_layers][T][n_q_heads][head_dim], 16-B aligned
  *  n_cached  keys before the new rows; n_cached + T <= capacity
- *  page      keys per page, a positive multiple of 128
+ *  page      keys per page, a positive multiple of 128 (the online merge makes
+ *            the result independent of it)
  *  out, lse  device fp32 [n_layers][T][n_q_heads][head_dim] and [...][n_q_heads]
- *  page_out, page_lse  optional (both NULL or both set): per-page partials
- *            [n_layers][T][n_q_heads][n_pages][head_dim] and [...][n_pages],
- *            n_pages = ceil((n_cached + T) / page)
- *  workspace device scratch of at least kvq_workspace_bytes(KVQ_OP_PREFILL,...)
- *            bytes (may be NULL when that is 0), 256-B aligned
- * Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED (head_dim != 256 or
- *         group size not dividing the 128-row tile), CUDA. */
+ *  page_out, page_lse  must be NULL: per-page partial outputs are not built
+ *            (both set -> KVQ_ERR_UNSUPPORTED)
+ *  workspace unused (kvq_workspace_bytes(KVQ_OP_PREFILL, ...) is 0); may be NULL
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (group size > 32, page outputs),
+ *         CUDA. */
 kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
                             int n_q_heads, int T, int64_t n_cached, int page, float scale,
                             float *out, float *lse, float *page_out, float *page_lse,

@@ -296,6 +296,7 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
     if (page_out) {
         KVQ_TRY(need(page_out, 16, "page_out", fn));
         KVQ_TRY(need(page_lse, 4, "page_lse", fn));
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: per-page partial outputs are not built", fn);
     }
     const int H = layers[0].n_kv_heads, D = layers[0].head_dim;
     if (n_q_heads < 1 || n_q_heads % H != 0)

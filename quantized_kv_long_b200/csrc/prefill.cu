@@ -1,12 +1,677 @@
-// prefill.cu -- chunked prefill attention (not yet built: reports unsupported).
+// prefill.cu -- chunked prefill attention over the Q8_0/Q4_0 cache.
+//
+// What it computes ("Online Log-Sum-Exp prefill & pipelined prefetch" of the
+// RX 9070 XT KV-streaming page: prefill computed chunk by chunk over streamed
+// pages of keys with the log-sum-exp accumulated online): T new query tokens
+// per layer, appended at rows [n_cached, n_cached + T), attend to keys
+// j <= n_cached + t (query token t); GQA: query head g reads KV head g / G.
+// out = sum_j p_j v^_j / l and lse = m + ln l over all visible keys, with the
+// online (running max, running sum) merge carried across pages of keys
+// inside the kernel.
+//
+// Two kernels:
+//  * prefill_tc_kernel -- the tensor-core path (tcgen05, TMEM) for rows that
+//    see at least PF_MIN_KEYS keys.  One CTA per (128 query rows of one KV
+//    head's group, KV head, layer); rows are (token, q head) pairs.  Per tile
+//    of 48 keys:
+//      - a producer warp bulk-copies the tile's raw Q8_0 K head-rows (48 x
+//        272 B) and Q4_0 V head-rows (48 x 144 B) into a 2-deep staging ring;
+//      - 8 dequant warps turn them into f16 tiles in shared memory with
+//        128-byte swizzle: K^ = d * q as an exact two-part f16 sum (K^hi =
+//        RN_f16(d q), K^lo = fma(d, q, -K^hi)), K-major (keys x head_dim), and
+//        V^ = RN_f16(d * (u - 8)) MN-major (keys x head_dim), zeros past the
+//        end;
+//      - one thread issues tcgen05.mma: S = Q K^hi^T + Q K^lo^T (A = Q held
+//        in tensor memory, M = 128, N = 48, K = 256, twice) into a double-
+//        buffered S in TMEM -- exact products, so the logits carry only fp32
+//        rounding -- then O += P V^ (A = P in TMEM, written over S; N = 256,
+//        K = 48) into the fp32 O accumulator in TMEM (256 columns);
+//      - 4 softmax warps own one query row per thread (its TMEM lane): they
+//        read S, apply the causal mask, keep a lazy running max (moves only
+//        when a score exceeds it by 8 in log2 units, with an exact rescale of
+//        O in TMEM) and write P = 2^(s - m) as f16 back into TMEM.
+//    V^ and P carry one f16 rounding each (relative 2^-11).  These errors are
+//    independent per key and average over the visible keys, but a row whose
+//    softmax is peaked (a large query component on an x8 outlier channel) can
+//    give one key a large share of the weight at a few thousand keys, and one
+//    f16 rounding of |v^| ~ 20 is ~1e-2; a rounded K^ would move that key's
+//    logit by ~2e-3 (why K^ is split exactly).  Measured max-abs error of this
+//    path against the oracle (96 sampled rows, N(0,1) K/V with x8 outlier
+//    channels): 4.7e-4 at 4,352 keys, 2.2e-4 at 16,384, 9.1e-5 at 65,536,
+//    8.8e-5 at 262,144 (tolerance 2e-3).  Rows that see fewer than
+//    PF_MIN_KEYS = 16,384 keys take the exact kernel.
+//  * prefill_exact_kernel -- CUDA cores, fp32 with per-block scaling (the
+//    same arithmetic as the general decode kernel), for rows that see fewer
+//    than PF_MIN_KEYS keys.
+// Every mbarrier wait is bounded; a wait that runs out records
+// KVQ_ERR_TIMEOUT in the status word and the roles fall through, waiting
+// (bounded) for their own copies and MMAs before the CTA frees TMEM and exits.
+#include <stdlib.h>
+
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace kvq {
 
+namespace {
+
+constexpr int PF_MIN_KEYS = 16384;
+constexpr int BM = 128, BN = 48, HD = 256;
+constexpr int KROW = 272, VROW = 144;
+constexpr int RAW_K = BN * KROW, RAW_V = BN * VROW, RAW_BYTES = RAW_K + RAW_V;
+constexpr int TILE_H = BN * HD * 2;  // one f16 tile of 48 keys x 256 dims: 24 KB
+constexpr int N_SOFT = 4, N_DEQ = 8;
+constexpr int W_PROD = N_SOFT + N_DEQ, W_MMA = W_PROD + 1;
+constexpr int PF_THREADS = (W_MMA + 1) * 32;  // 14 warps
+constexpr uint64_t WAIT_NS = 1000000000ull;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+constexpr float TAU = 8.0f;
+constexpr float M_INIT = -1.0e30f;
+// tensor-memory columns
+constexpr uint32_t COL_O = 0, COL_Q = 256, COL_S0 = 384;  // S buffer b at COL_S0 + BN b
+
+struct PfSmemHead {
+    uint64_t raw_full[2], raw_free[2], kv_full[2], s_full[2], p_full[2], pv_done[2], q_ready;
+    uint32_t tmem_base;
+    int abort;
+};
+// layout: [K^hi 2 x 24K][K^lo 2 x 24K][V^ 2 x 24K][raw 2 x 19,968][head], base 1024-aligned
+constexpr int OFF_KH = 0, OFF_KL = 2 * TILE_H, OFF_VH = 4 * TILE_H, OFF_RAW = 6 * TILE_H;
+constexpr int OFF_HEAD = OFF_RAW + 2 * RAW_BYTES;
+constexpr int PF_SMEM = OFF_HEAD + (int)sizeof(PfSmemHead) + 1024;  // + alignment slack
+
+// byte offset of (row, dim) in a [BN rows x 256 dims] f16 tile stored as four
+// 1024-aligned column blocks of [BN rows x 128 B] with the 128-byte swizzle
+__device__ __forceinline__ uint32_t sw_off(int row, int dim)
+{
+    const int c16 = (dim >> 3) & 7;
+    return (uint32_t)((dim >> 6) * (BN * 128) + row * 128 + ((c16 ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t lds32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+__device__ __forceinline__ uint32_t lds16(const uint8_t *p) { return *reinterpret_cast<const uint16_t *>(p); }
+
+__device__ __forceinline__ __half2 dup_h(uint32_t d16)
+{
+    return ptx::bits_h2(d16 | (d16 << 16));
+}
+
+// four int8 -> d * q as an exact two-part f16 sum: x = RN(d q) (two half2) and
+// r = d q - x = fma(d, q, -x) (exact: q has 8 significant bits, d 11)
+__device__ __forceinline__ void k4(uint32_t w, __half2 d2, uint32_t (&x)[2], uint32_t (&r)[2])
+{
+    w ^= 0x80808080u;
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+    const __half2 a = __hsub2(ptx::bits_h2(ptx::prmt(w, 0x64646464u, 0x5140)), bias);
+    const __half2 b = __hsub2(ptx::bits_h2(ptx::prmt(w, 0x64646464u, 0x7362)), bias);
+    const __half2 xa = __hmul2_rn(a, d2), xb = __hmul2_rn(b, d2);
+    x[0] = ptx::h2_bits(xa);
+    x[1] = ptx::h2_bits(xb);
+    r[0] = ptx::h2_bits(__hfma2(a, d2, __hneg2(xa)));
+    r[1] = ptx::h2_bits(__hfma2(b, d2, __hneg2(xb)));
+}
+
+// two Q4_0 bytes (at bits 0-7 and 16-23 of x) -> low-nibble and high-nibble half2, times d
+__device__ __forceinline__ void v2(uint32_t x, __half2 d2, uint32_t &lo, uint32_t &hi)
+{
+    const __half2 c1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+    const __half2 s16 = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+    const __half2 c72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
+    const __half2 a = __hsub2(ptx::bits_h2((x & 0x000F000Fu) | 0x64006400u), c1032);
+    const __half2 b = __hfma2(ptx::bits_h2((x & 0x00F000F0u) | 0x64006400u), s16, c72);
+    lo = ptx::h2_bits(__hmul2_rn(a, d2));
+    hi = ptx::h2_bits(__hmul2_rn(b, d2));
+}
+
+__device__ __forceinline__ void sts128(uint8_t *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
+}
+
+__global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const PrefillArgs a, int row0)
+{
+    extern __shared__ __align__(1024) uint8_t pf_raw[];
+    uint8_t *smem = pf_raw + ((1024u - (ptx::smem_u32(pf_raw) & 1023u)) & 1023u);
+    PfSmemHead &hd = *reinterpret_cast<PfSmemHead *>(smem + OFF_HEAD);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int rows_total = a.T * G;
+    const int h = blockIdx.y, layer = blockIdx.z;
+    const int R0 = row0 + blockIdx.x * BM;                 // first row of this tile
+    const int r_last = min(R0 + BM, rows_total) - 1;
+    const int64_t n_keys = a.n_cached + r_last / G + 1;    // keys any row of the tile sees
+    const int ntiles = (int)((n_keys + BN - 1) / BN);
+    const int64_t cap = a.layers.cap[layer];
+    const uint8_t *kg = a.layers.k[layer] + (int64_t)h * cap * KROW;
+    const uint8_t *vg = a.layers.v[layer] + (int64_t)h * cap * VROW;
+    volatile int *abort = &hd.abort;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&hd.raw_full[i], 1);
+            ptx::mbar_init(&hd.raw_free[i], N_DEQ);
+            ptx::mbar_init(&hd.kv_full[i], N_DEQ);
+            ptx::mbar_init(&hd.s_full[i], 1);
+            ptx::mbar_init(&hd.p_full[i], N_SOFT);
+            ptx::mbar_init(&hd.pv_done[i], 1);
+        }
+        ptx::mbar_init(&hd.q_ready, N_SOFT);
+        hd.abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == W_MMA) {
+        ptx::tmem_alloc(&hd.tmem_base, 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tbase = hd.tmem_base;
+    auto fail = [&]() {
+        if (!*abort) {
+            *abort = 1;
+            report_timeout(a.status);
+        }
+    };
+
+    if (warp < N_SOFT) {
+        // ================================================================ softmax
+        const int i = warp * 32 + lane;  // query row of this thread = its TMEM lane
+        const int gr = R0 + i;
+        const bool live = gr <= r_last;
+        const int t = live ? gr / G : 0, gq = live ? gr % G : 0;
+        const int64_t lim = a.n_cached + t;  // last visible key
+        const uint32_t lane_addr = tbase + ((uint32_t)(warp * 32) << 16);
+        {   // Q row -> TMEM columns [COL_Q, COL_Q + 128): two f16 per column, lower dim low
+            const uint4 *qp = reinterpret_cast<const uint4 *>(
+                a.q + (((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq) * HD);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t r[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 x = live ? qp[c * 4 + v] : make_uint4(0u, 0u, 0u, 0u);
+                    r[4 * v + 0] = x.x;
+                    r[4 * v + 1] = x.y;
+                    r[4 * v + 2] = x.z;
+                    r[4 * v + 3] = x.w;
+                }
+                ptx::tmem_st16(lane_addr + COL_Q + 16 * c, r);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                ptx::mbar_arrive(&hd.q_ready);
+        }
+        const float sl2 = a.scale * LOG2E;
+        float m = M_INIT, l = 0.0f;
+        for (int j = 0; j < ntiles; ++j) {
+            const int b = j & 1;
+            const uint32_t scol = COL_S0 + BN * b;
+            bool ok = true;
+            if (lane == 0)
+                ok = ptx::mbar_wait_bounded(&hd.s_full[b], (j >> 1) & 1, abort, WAIT_NS);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                if (lane == 0)
+                    fail();
+                break;
+            }
+            ptx::tc_fence_after();
+            float s[BN];
+#pragma unroll
+            for (int c = 0; c < BN / 16; ++c) {
+                uint32_t r[16];
+                ptx::tmem_ld16(lane_addr + scol + 16 * c, r);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    s[16 * c + e] = __uint_as_float(r[e]) * sl2;
+            }
+            const int64_t kj0 = (int64_t)j * BN;
+            if (kj0 + BN - 1 > lim) {  // causal edge / end of the keys
+#pragma unroll
+                for (int e = 0; e < BN; ++e)
+                    if (kj0 + e > lim)
+                        s[e] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int e = 1; e < BN; ++e)
+                mx = fmaxf(mx, s[e]);
+            float alpha = 1.0f;
+            if (mx > m + TAU) {
+                alpha = ptx::ex2(m - mx);
+                m = mx;
+                l *= alpha;
+            }
+            // rescale O (rare): the whole warp takes part once any lane needs it
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                bool okp = true;
+                if (lane == 0)
+                    okp = ptx::mbar_wait_bounded(&hd.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1,
+                                                 abort, WAIT_NS);
+                if (!__shfl_sync(0xffffffffu, okp ? 1 : 0, 0)) {
+                    if (lane == 0)
+                        fail();
+                    break;
+                }
+                ptx::tc_fence_after();
+                for (int c = 0; c < 16; ++c) {
+                    uint32_t r[16];
+                    ptx::tmem_ld16(lane_addr + COL_O + 16 * c, r);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                    ptx::tmem_st16(lane_addr + COL_O + 16 * c, r);
+                }
+                ptx::tmem_wait_st();
+            }
+            // P = 2^(s - m) in f16 over the first BN/2 columns of this S buffer
+            uint32_t pk[BN / 2 + 8];
+#pragma unroll
+            for (int e = 0; e < BN / 2; ++e) {
+                const float p0 = ptx::ex2(s[2 * e] - m), p1 = ptx::ex2(s[2 * e + 1] - m);
+                l += p0 + p1;
+                pk[e] = ptx::h2_bits(__floats2half2_rn(p0, p1));
+            }
+            ptx::tmem_st16(lane_addr + scol, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+            // the last 8 P columns (keys 32..47); the 8 columns after them belong to
+            // this S buffer too and are rewritten by the next QK^T
+#pragma unroll
+            for (int e = BN / 2; e < BN / 2 + 8; ++e)
+                pk[e] = 0u;
+            ptx::tmem_st16(lane_addr + scol + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                ptx::mbar_arrive(&hd.p_full[b]);
+        }
+        // ---- epilogue: out = O / l, lse = (m + log2 l) ln 2
+        if (!*abort) {
+            const int last = ntiles - 1;
+            bool ok = true;
+            if (lane == 0)
+                ok = ptx::mbar_wait_bounded(&hd.pv_done[last & 1], (last >> 1) & 1, abort, WAIT_NS);
+            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                ptx::tc_fence_after();
+                const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+                float4 *op = reinterpret_cast<float4 *>(
+                    a.out + (((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq) * HD);
+                for (int c = 0; c < 16; ++c) {
+                    uint32_t r[16];
+                    ptx::tmem_ld16(lane_addr + COL_O + 16 * c, r);
+                    ptx::tmem_wait_ld();
+                    if (live) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            op[c * 4 + v] = make_float4(__uint_as_float(r[4 * v]) * inv,
+                                                        __uint_as_float(r[4 * v + 1]) * inv,
+                                                        __uint_as_float(r[4 * v + 2]) * inv,
+                                                        __uint_as_float(r[4 * v + 3]) * inv);
+                    }
+                }
+                if (live)
+                    a.lse[((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq] =
+                        l > 0.0f ? (m + log2f(l)) * LN2 : -INFINITY;
+            } else if (lane == 0) {
+                fail();
+            }
+        }
+    } else if (warp < W_PROD) {
+        // ================================================================ dequant
+        const int dt = threadIdx.x - N_SOFT * 32;  // 0..255
+        for (int j = 0; j < ntiles; ++j) {
+            const int b = j & 1;
+            bool ok = true;
+            if (lane == 0)
+                ok = ptx::mbar_wait_bounded(&hd.raw_full[b], (j >> 1) & 1, abort, WAIT_NS) &&
+                     ptx::mbar_wait_bounded(&hd.pv_done[b], ((j >> 1) & 1) ^ 1, abort, WAIT_NS);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                if (lane == 0)
+                    fail();
+                break;
+            }
+            const int rows = (int)min((int64_t)BN, n_keys - (int64_t)j * BN);
+            const uint8_t *rk = smem + OFF_RAW + b * RAW_BYTES;
+            const uint8_t *rv = rk + RAW_K;
+            uint8_t *kh = smem + OFF_KH + b * TILE_H;
+            uint8_t *kl = smem + OFF_KL + b * TILE_H;
+            uint8_t *vh = smem + OFF_VH + b * TILE_H;
+#pragma unroll 1
+            for (int u = dt; u < BN * 8; u += N_DEQ * 32) {
+                const int r = u >> 3, bk = u & 7;
+                uint32_t w[8];
+                if (r < rows) {
+                    // ---- K block: d (fp16) + 32 int8
+                    const uint8_t *src = rk + r * KROW + 34 * bk;
+                    uint32_t d16;
+                    if ((bk & 1) == 0) {  // block starts 4-byte aligned: d, q0, q1 | ...
+                        uint32_t x[9];
+#pragma unroll
+                        for (int i = 0; i < 9; ++i)
+                            x[i] = lds32(src + 4 * i);
+                        d16 = x[0] & 0xFFFFu;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            w[i] = ptx::prmt(x[i], x[i + 1], 0x5432);
+                    } else {              // qs start 4-byte aligned
+                        d16 = lds16(src);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            w[i] = lds32(src + 2 + 4 * i);
+                    }
+                    const __half2 d2 = dup_h(d16);
+#pragma unroll
+                    for (int m4 = 0; m4 < 4; ++m4) {
+                        uint32_t x0[2], x1[2], r0[2], r1[2];
+                        k4(w[2 * m4], d2, x0, r0);
+                        k4(w[2 * m4 + 1], d2, x1, r1);
+                        sts128(kh + sw_off(r, 32 * bk + 8 * m4), x0[0], x0[1], x1[0], x1[1]);
+                        sts128(kl + sw_off(r, 32 * bk + 8 * m4), r0[0], r0[1], r1[0], r1[1]);
+                    }
+                    // ---- V block: d (fp16) + 16 bytes of nibbles
+                    const uint8_t *vsrc = rv + r * VROW + 18 * bk;
+                    uint32_t vw[4];
+                    if ((bk & 1) == 0) {
+                        uint32_t x[5];
+#pragma unroll
+                        for (int i = 0; i < 5; ++i)
+                            x[i] = lds32(vsrc + 4 * i);
+                        d16 = x[0] & 0xFFFFu;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            vw[i] = ptx::prmt(x[i], x[i + 1], 0x5432);
+                    } else {
+                        d16 = lds16(vsrc);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            vw[i] = lds32(vsrc + 2 + 4 * i);
+                    }
+                    const __half2 dv = dup_h(d16);
+                    // byte j of the block: element j (low nibble), element j + 16 (high)
+                    uint32_t lo[8], hi[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        v2(ptx::prmt(vw[i], 0u, 0x4140), dv, lo[2 * i], hi[2 * i]);      // bytes 0, 1
+                        v2(ptx::prmt(vw[i], 0u, 0x4342), dv, lo[2 * i + 1], hi[2 * i + 1]);  // bytes 2, 3
+                    }
+                    sts128(vh + sw_off(r, 32 * bk + 0), lo[0], lo[1], lo[2], lo[3]);
+                    sts128(vh + sw_off(r, 32 * bk + 8), lo[4], lo[5], lo[6], lo[7]);
+                    sts128(vh + sw_off(r, 32 * bk + 16), hi[0], hi[1], hi[2], hi[3]);
+                    sts128(vh + sw_off(r, 32 * bk + 24), hi[4], hi[5], hi[6], hi[7]);
+                } else {
+                    // keys past the end: zero K and V so that 0-weight products stay 0
+#pragma unroll
+                    for (int m4 = 0; m4 < 4; ++m4) {
+                        sts128(kh + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
+                        sts128(kl + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
+                        sts128(vh + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
+                    }
+                }
+            }
+            ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(&hd.raw_free[b]);
+                ptx::mbar_arrive(&hd.kv_full[b]);
+            }
+        }
+    } else if (warp == W_PROD) {
+        // ================================================================ copies
+        if (lane == 0) {
+            int issued = 0;
+            for (int j = 0; j < ntiles; ++j) {
+                const int b = j & 1;
+                if (*abort ||
+                    !ptx::mbar_wait_bounded(&hd.raw_free[b], ((j >> 1) & 1) ^ 1, abort, WAIT_NS) ||
+                    (j >= 2 && !ptx::mbar_wait_bounded(&hd.raw_full[b], ((j >> 1) - 1) & 1, abort,
+                                                       WAIT_NS))) {
+                    fail();
+                    break;
+                }
+                const int rows = (int)min((int64_t)BN, n_keys - (int64_t)j * BN);
+                uint8_t *dst = smem + OFF_RAW + b * RAW_BYTES;
+                ptx::mbar_arrive_expect_tx(&hd.raw_full[b], rows * (KROW + VROW));
+                ptx::bulk_g2s(dst, kg + (int64_t)j * RAW_K, rows * KROW, &hd.raw_full[b]);
+                ptx::bulk_g2s(dst + RAW_K, vg + (int64_t)j * RAW_V, rows * VROW, &hd.raw_full[b]);
+                issued = j + 1;
+            }
+            int none = 0;
+            for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
+                if (!ptx::mbar_wait_bounded(&hd.raw_full[j & 1], (j >> 1) & 1, &none, WAIT_NS))
+                    report_timeout(a.status);
+        }
+    } else {
+        // ================================================================ MMA issue
+        if (lane == 0) {
+            const uint32_t id_qk = ptx::idesc_f16_f32(BM, BN, false, false);
+            const uint32_t id_pv = ptx::idesc_f16_f32(BM, HD, false, true);
+            int committed = -1;  // last tile whose PV was committed
+            bool ok = ptx::mbar_wait_bounded(&hd.q_ready, 0, abort, WAIT_NS);
+            auto issue_pv = [&](int jj) -> bool {
+                const int bb = jj & 1;
+                if (!ptx::mbar_wait_bounded(&hd.p_full[bb], (jj >> 1) & 1, abort, WAIT_NS))
+                    return false;
+                ptx::tc_fence_after();
+                const uint8_t *vh = smem + OFF_VH + bb * TILE_H;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    ptx::umma_f16_ts(tbase + COL_O, tbase + COL_S0 + BN * bb + 8 * kk,
+                                     ptx::smem_desc_sw128(vh + kk * 2 * 1024, BN * 128, 1024), id_pv,
+                                     jj > 0 || kk > 0);
+                ptx::umma_commit(&hd.pv_done[bb]);
+                committed = jj;
+                return true;
+            };
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int b = j & 1;
+                ok = ptx::mbar_wait_bounded(&hd.kv_full[b], (j >> 1) & 1, abort, WAIT_NS) &&
+                     (j < 2 || ptx::mbar_wait_bounded(&hd.pv_done[b], ((j >> 1) - 1) & 1, abort,
+                                                       WAIT_NS));
+                if (!ok)
+                    break;
+                ptx::tc_fence_after();
+                // S = Q K^hi^T + Q K^lo^T: exact products of q and d*q_int, fp32 sums
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint8_t *kt = smem + (part ? OFF_KL : OFF_KH) + b * TILE_H;
+#pragma unroll
+                    for (int ks = 0; ks < HD / 16; ++ks)
+                        ptx::umma_f16_ts(tbase + COL_S0 + BN * b, tbase + COL_Q + 8 * ks,
+                                         ptx::smem_desc_sw128(kt + (ks >> 2) * (BN * 128) + (ks & 3) * 32,
+                                                              16, 1024),
+                                         id_qk, part > 0 || ks > 0);
+                }
+                ptx::umma_commit(&hd.s_full[b]);
+                if (j >= 1)
+                    ok = issue_pv(j - 1);
+            }
+            if (ok)
+                ok = issue_pv(ntiles - 1);
+            if (!ok)
+                fail();
+            // every committed MMA has finished before TMEM is freed
+            int none = 0;
+            if (committed >= 0 &&
+                !ptx::mbar_wait_bounded(&hd.pv_done[committed & 1], (committed >> 1) & 1, &none,
+                                        WAIT_NS))
+                report_timeout(a.status);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == W_MMA) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tbase, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Exact path for short visible ranges: one CTA per (token block, KV head,
+// layer); rows (t, g) of TB tokens; keys in tiles of 64 with an online
+// softmax in fp32; per-block K scale applied to each block's fp32 dot product.
+constexpr int EX_THREADS = 256, EX_TILE = 64;
+
+__global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const PrefillArgs a, int tb_tok,
+                                                                   int t_end)
+{
+    extern __shared__ float ex_sm[];
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int D = a.head_dim, nb = D / QK;
+    const int t0 = blockIdx.x * tb_tok;
+    const int ntok = min(tb_tok, t_end - t0);
+    const int R = ntok * G;
+    const int h = blockIdx.y, layer = blockIdx.z;
+    float *q_s = ex_sm;                 // [R][D]
+    float *acc = q_s + R * D;           // [R][D]
+    float *p_s = acc + R * D;           // [R][TILE]
+    float *m_s = p_s + R * EX_TILE;
+    float *l_s = m_s + R;
+    float *al_s = l_s + R;
+    const uint8_t *kb = a.layers.k[layer] + (int64_t)h * a.layers.cap[layer] * k_row_bytes(D);
+    const uint8_t *vb = a.layers.v[layer] + (int64_t)h * a.layers.cap[layer] * v_row_bytes(D);
+    for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
+        const int r = p / D, i = p % D;
+        const int t = t0 + r / G, g = r % G;
+        q_s[p] = __half2float(a.q[(((int64_t)layer * a.T + t) * a.n_q_heads + h * G + g) * D + i]);
+        acc[p] = 0.0f;
+    }
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+        m_s[r] = -INFINITY;
+        l_s[r] = 0.0f;
+    }
+    __syncthreads();
+    const int64_t kend = a.n_cached + t0 + ntok;  // keys the last token sees
+    for (int64_t j0 = 0; j0 < kend; j0 += EX_TILE) {
+        for (int p = threadIdx.x; p < R * EX_TILE; p += blockDim.x) {
+            const int r = p / EX_TILE, jj = p % EX_TILE;
+            const int64_t j = j0 + jj;
+            const int t = t0 + r / G;
+            float s = -INFINITY;
+            if (j <= a.n_cached + t) {
+                const uint8_t *kr = kb + j * k_row_bytes(D);
+                const float *qr = q_s + r * D;
+                float tot = 0.0f;
+                for (int bq = 0; bq < nb; ++bq) {
+                    const uint8_t *blk = kr + bq * Q8_0_BYTES;
+                    const float d = __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
+                    float part = 0.0f;
+                    for (int i = 0; i < QK; ++i)
+                        part += qr[bq * QK + i] * (float)(int8_t)blk[2 + i];
+                    tot += d * part;
+                }
+                s = a.scale * tot;
+            }
+            p_s[p] = s;
+        }
+        __syncthreads();
+        for (int r = threadIdx.x; r < R; r += blockDim.x) {
+            float mt = -INFINITY;
+            for (int jj = 0; jj < EX_TILE; ++jj)
+                mt = fmaxf(mt, p_s[r * EX_TILE + jj]);
+            const float m_old = m_s[r], m_new = fmaxf(m_old, mt);
+            float alpha = 1.0f, sum = 0.0f;
+            if (m_new != -INFINITY) {
+                alpha = (m_old == -INFINITY) ? 0.0f : expf(m_old - m_new);
+                for (int jj = 0; jj < EX_TILE; ++jj) {
+                    const float s = p_s[r * EX_TILE + jj];
+                    const float pw = (s == -INFINITY) ? 0.0f : expf(s - m_new);
+                    p_s[r * EX_TILE + jj] = pw;
+                    sum += pw;
+                }
+            } else {
+                for (int jj = 0; jj < EX_TILE; ++jj)
+                    p_s[r * EX_TILE + jj] = 0.0f;
+            }
+            l_s[r] = l_s[r] * alpha + sum;
+            m_s[r] = m_new;
+            al_s[r] = alpha;
+        }
+        __syncthreads();
+        for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
+            const int r = p / D, i = p % D;
+            const int bq = i / QK, ii = i % QK;
+            float o = acc[p] * al_s[r];
+            for (int jj = 0; jj < EX_TILE; ++jj) {
+                const float pw = p_s[r * EX_TILE + jj];
+                if (pw == 0.0f)
+                    continue;
+                const uint8_t *blk = vb + (j0 + jj) * v_row_bytes(D) + bq * Q4_0_BYTES;
+                const float d = __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
+                const uint8_t byte = blk[2 + (ii & 15)];
+                const int u = ii < 16 ? (byte & 15) : (byte >> 4);
+                o += pw * (d * (float)(u - 8));
+            }
+            acc[p] = o;
+        }
+        __syncthreads();
+    }
+    for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
+        const int r = p / D, i = p % D;
+        const int t = t0 + r / G, g = r % G;
+        const int64_t row = ((int64_t)layer * a.T + t) * a.n_q_heads + h * G + g;
+        const float l = l_s[r];
+        a.out[row * D + i] = (l > 0.0f) ? acc[p] / l : 0.0f;
+        if (i == 0)
+            a.lse[row] = (l > 0.0f) ? m_s[r] + logf(l) : -INFINITY;
+    }
+}
+
+}  // namespace
+
 size_t prefill_workspace_bytes(int, int, int, int, int) { return 0; }
 
-bool prefill_supported(int, int, int) { return false; }
+bool prefill_supported(int n_q_heads, int n_kv_heads, int head_dim)
+{
+    const int G = n_q_heads / n_kv_heads;
+    return G >= 1 && G <= 32 && head_dim >= 32 && head_dim <= 512 && head_dim % 32 == 0;
+}
 
-void launch_prefill(const PrefillArgs &, cudaStream_t) {}
+void launch_prefill(const PrefillArgs &a, cudaStream_t s)
+{
+    const int G = a.n_q_heads / a.n_kv_heads;
+    // tokens whose rows see fewer than PF_MIN_KEYS keys take the exact kernel
+    // (host test hook KVQ_PREFILL_TC_MIN_KEYS moves the threshold)
+    int64_t min_keys = PF_MIN_KEYS;
+    if (const char *e = getenv("KVQ_PREFILL_TC_MIN_KEYS"))
+        min_keys = atoll(e);
+    int64_t t_split = min_keys - 1 - a.n_cached;
+    t_split = t_split < 0 ? 0 : (t_split > a.T ? a.T : t_split);
+    if (a.head_dim != HD)
+        t_split = a.T;  // the tensor-core path is built for head_dim 256
+    if (t_split > 0) {
+        const int tb = max(1, 32 / G);
+        const size_t smem = sizeof(float) * ((size_t)2 * tb * G * a.head_dim +
+                                             (size_t)tb * G * EX_TILE + 3 * (size_t)tb * G);
+        static bool attr_ex[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (smem > 48 * 1024 && dev >= 0 && dev < 64 && !attr_ex[dev]) {
+            cudaFuncSetAttribute(prefill_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+            attr_ex[dev] = true;
+        }
+        dim3 grid((unsigned)((t_split + tb - 1) / tb), a.n_kv_heads, a.n_layers);
+        prefill_exact_kernel<<<grid, EX_THREADS, smem, s>>>(a, tb, (int)t_split);
+    }
+    if (t_split < a.T) {
+        static bool attr_tc[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 0 && dev < 64 && !attr_tc[dev]) {
+            cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 PF_SMEM);
+            attr_tc[dev] = true;
+        }
+        const int row0 = (int)t_split * G;
+        const int rows = a.T * G - row0;
+        dim3 grid((unsigned)((rows + BM - 1) / BM), a.n_kv_heads, a.n_layers);
+        prefill_tc_kernel<<<grid, PF_THREADS, PF_SMEM, s>>>(a, row0);
+    }
+}
 
 }  // namespace kvq

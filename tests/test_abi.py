@@ -129,6 +129,7 @@ def test_prefill_validation(kvq):
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, page=100)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, n_cached=4000)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, page_out=A)
+    _raises(kvq, kvq.KVQ_ERR_UNSUPPORTED, call, page_out=A, page_lse=A)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, T=0)
     _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, call, out=A + 4)
 

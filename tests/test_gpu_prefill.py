@@ -1,0 +1,97 @@
+"""Chunked prefill on the GPU against the oracle.
+
+Cases cover the tensor-core path (every row sees >= 4,096 keys), the exact
+path (short prompts), a run that splits between them, ragged row tiles, several
+layers per call, and the full prefill262k workload (2,048 new tokens over
+262,144 cached, 16 layers in one call) on sampled rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_kv_long_b200 import workload as wl
+
+from helpers import assert_attn_close, fill_both
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from quantized_kv_long_b200 import kvq as m
+    return m
+
+
+def run_prefill(kvq, cache, q, Hq, T, n_cached, scale, page=1024):
+    L, D = q.shape[0], q.shape[-1]
+    out = torch.full((L, T, Hq, D), float("nan"), device="cuda")
+    lse = torch.full((L, T, Hq), float("nan"), device="cuda")
+    kvq.kvq_prefill_attn(cache.layers(), torch.from_numpy(q).cuda(), Hq, T, n_cached, page, scale,
+                         out, lse)
+    kvq.kvq_check()
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+def check(kvq, w, n_layers, T, n_cached):
+    n = n_cached + T
+    cap = -(-n // 8) * 8
+    layers = list(range(n_layers))
+    cache, orc = fill_both(w, layers, n, cap)
+    q = np.stack([wl.q_rows(w, l, T) for l in layers])
+    out, lse = run_prefill(kvq, cache, q, w.n_q_heads, T, n_cached, w.scale)
+    for l in layers:
+        ro, rl = oracle.prefill_attn(orc[l][0], orc[l][1], q[l], n_cached, 1024, w.scale)
+        assert_attn_close(out[l], lse[l], ro, rl, f"prefill layer {l}")
+
+
+def test_tensor_core_path(kvq):
+    """Every row sees >= 16,448 keys; 128 tokens x 6 heads = 6 full 128-row tiles per head."""
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=16448, T=128)
+    check(kvq, w, 1, 128, 16448)
+
+
+def test_split_exact_and_tensor_core_ragged(kvq):
+    """Tokens 0..85 see < 16,384 keys (exact kernel), 86..299 take the tensor
+    cores; 214 x 6 rows of the tensor-core part leave a ragged last tile."""
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=16298, T=300)
+    check(kvq, w, 2, 300, 16298)
+
+
+def test_short_prompt_exact(kvq):
+    """No cached keys: token 0 sees exactly one key (the exact kernel)."""
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=0, T=70)
+    check(kvq, w, 1, 70, 0)
+
+
+def test_exact_kernel_layers(kvq):
+    """Mid-length context on the exact kernel, three layers in one call."""
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=9000, T=40)
+    check(kvq, w, 3, 40, 9000)
+
+
+def test_prefill262k_full_size_sampled(kvq):
+    """The full workload in the launch configuration the benchmark times:
+    16 layers, 2,048 new tokens appended after 262,144 cached keys."""
+    import bench
+    w = wl.WORKLOADS["prefill262k"]
+    T, nc, Hq = w.T, w.n_cached, w.n_q_heads
+    device = torch.device("cuda", 0)
+    cache = bench.fill_cache(kvq, torch, wl.small(w, n_kv=nc + T), device)
+    q = np.stack([wl.q_rows(w, l) for l in range(w.n_layers)])
+    out = torch.full((w.n_layers, T, Hq, 256), float("nan"), device=device)
+    lse = torch.full((w.n_layers, T, Hq), float("nan"), device=device)
+    kvq.kvq_prefill_attn(cache.layers(), torch.from_numpy(q).cuda(), Hq, T, nc, w.page, w.scale,
+                         out, lse)
+    kvq.kvq_check()
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    rng = np.random.default_rng(7)
+    for l in (0, 9):
+        kc, vc = oracle.empty_cache(w.n_kv_heads, w.head_dim, nc + T)
+        oracle.append(kc, vc, wl.kv_rows(w, l, 0, 0, nc + T), wl.kv_rows(w, l, 1, 0, nc + T), 0)
+        ts = np.concatenate([[0, 1, T - 1], rng.integers(0, T, 9)])
+        hs = rng.integers(0, Hq, len(ts))
+        ro, rl = oracle.attn_rows(kc, vc, q[l, ts, hs], hs, Hq, np.zeros(len(ts)), nc + ts + 1,
+                                  w.scale)
+        assert_attn_close(out[l, ts, hs].cpu().numpy(), lse[l, ts, hs].cpu().numpy(), ro, rl,
+                          f"prefill262k layer {l}")
