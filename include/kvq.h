@@ -254,6 +254,39 @@ kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_layers,
                              kvq_stream copy);
 
 /* ---------------------------------------------------------------------- */
+/* Decode + merge without caller-provided scratch                          */
+/* ---------------------------------------------------------------------- */
+
+/* Size of the library's own device array for chunk partials (8 MiB). */
+#define KVQ_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* kvq_decode_attn followed by kvq_merge_lse, for callers that cannot allocate
+ * device memory for the chunk partials -- for example a plug-in inside a host
+ * program that owns all device memory and passes only inputs and outputs, or
+ * a step loop where a cudaMalloc (which may synchronise the device or fail
+ * under memory pressure) is not allowed.  The pages have no counterpart: this
+ * entry point exists for such callers only.
+ * The partials live in one 8 MiB array inside the library (a __device__
+ * object that every GPU which loads the library keeps until the process
+ * exits); the call itself allocates nothing.  Its first call on a device looks
+ * the array's address up (cudaGetSymbolAddress) with that device current; make
+ * that first call before capturing any stream.  All calls share the array and
+ * it keeps the last call's contents: the decode rewrites every partial it
+ * reads, so nothing needs clearing, but calls whose work overlaps on the GPU
+ * (on different streams, or different threads) race on it -- order them.
+ *  layers, q, n_q_heads, T, n_kv, chunk, scale  as kvq_decode_attn
+ *  out   device fp32 [n_layers][T][n_q_heads][head_dim], 16-B aligned
+ *  lse   device fp32 [n_layers][T][n_q_heads]
+ * Limit: n_layers * T * n_q_heads * ceil(n_kv / chunk) * (head_dim + 1) * 4
+ * bytes (rounded up) must fit in KVQ_STATIC_SCRATCH_BYTES -- e.g. one layer of
+ * the 262,144-key verify batch, or 16 layers at 65,536 keys with chunk 4,096.
+ * Errors: those of kvq_decode_attn and kvq_merge_lse; UNSUPPORTED when the
+ * partials exceed the array. */
+kvq_status kvq_decode_merged_static(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                                    int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                                    float *out, float *lse, kvq_stream stream);
+
+/* ---------------------------------------------------------------------- */
 /* Housekeeping                                                            */
 /* ---------------------------------------------------------------------- */
 

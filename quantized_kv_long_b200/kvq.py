@@ -38,6 +38,7 @@ KVQ_OP_DECODE = 1
 KVQ_OP_PREFILL = 2
 KVQ_MAX_LAYERS = 64
 KVQ_MAX_DECODE_T = 4
+KVQ_STATIC_SCRATCH_BYTES = 8 << 20
 
 QK, Q8_0_BYTES, Q4_0_BYTES = 32, 34, 18
 
@@ -66,6 +67,8 @@ _SIGS = {
                           _P], _I32),
     "kvq_stream_decode": ([_LP, _I32, _LP, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P,
                            _P], _I32),
+    "kvq_decode_merged_static": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P],
+                                 _I32),
     "kvq_workspace_bytes": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "kvq_check": ([_P], _I32),
     "kvq_status_string": ([_I32], ctypes.c_char_p),
@@ -171,6 +174,15 @@ def kvq_stream_decode(host_layers, dev_slots, q, n_q_heads: int, T: int, n_kv: i
     _check(_lib.kvq_stream_decode(harr, n, sarr, _ptr(q), n_q_heads, T, n_kv, chunk, scale,
                                   _ptr(out_part), _ptr(lse_part), _ptr(out), _ptr(lse),
                                   _stream(compute), _stream(copy)))
+
+
+def kvq_decode_merged_static(layers, q, n_q_heads: int, T: int, n_kv: int, chunk: int,
+                             scale: float, out, lse, stream=None) -> None:
+    """Decode + merge with the chunk partials in the library's own static device
+    array (for callers that cannot allocate); see include/kvq.h for the limit."""
+    arr, n = _layers(layers)
+    _check(_lib.kvq_decode_merged_static(arr, n, _ptr(q), n_q_heads, T, n_kv, chunk, scale,
+                                         _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def kvq_workspace_bytes(op: int, n_layers: int, n_q_heads: int, n_kv_heads: int, T: int,
