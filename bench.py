@@ -317,6 +317,108 @@ def run_ours(args, w: wl.Workload) -> dict | None:
 
 
 DECODE_SOURCES = ("decode.cu", "ptx.cuh", "common.cuh")
+STREAM_METRIC = "q8_0/q4_0 host-streamed decode: H2D GB/s (% of measured H2D), query-tok/s at 262k ctx"
+
+
+def h2d_peak(torch, device, nbytes: int) -> float:
+    """Best-of-5 pinned host -> device copy bandwidth (GB/s) of an nbytes buffer."""
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    best = 0.0
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize(device)
+        best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+    return best
+
+
+def run_stream(args, w: wl.Workload) -> dict | None:
+    """The stream262k step: the 16-layer cache lives in pinned host memory; every
+    layer is copied into one of two device slots while the previous layer's
+    decode attention + merge run on the other (kvq_stream_decode)."""
+    import torch
+    import torch.distributed as dist
+    from quantized_kv_long_b200 import kvq
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    compute = torch.cuda.current_stream(device)
+    copy = torch.cuda.Stream(device)
+    L, T, Hq, D, n_kv, chunk = w.n_layers, w.T, w.n_q_heads, w.head_dim, w.n_kv, w.chunk
+    C = w.n_chunks
+    host = kvq.QuantizedKVCache(L, w.n_kv_heads, D, w.capacity, device="cpu", pin=True)
+    tmp = kvq.QuantizedKVCache(1, w.n_kv_heads, D, w.capacity, device=device)
+    for l in range(L):  # quantize on the GPU, keep the cache on the host
+        for start in range(0, n_kv, 131072):
+            stop = min(n_kv, start + 131072)
+            k = torch.from_numpy(wl.kv_rows(w, l, 0, start, stop)).to(device)
+            v = torch.from_numpy(wl.kv_rows(w, l, 1, start, stop)).to(device)
+            kvq.kvq_append(tmp.layer(0), k, v, start, stop - start)
+        host.k[l].copy_(tmp.k[0])
+        host.v[l].copy_(tmp.v[0])
+    del tmp
+    slots = kvq.QuantizedKVCache(2, w.n_kv_heads, D, w.capacity, device=device)
+    q = torch.from_numpy(np.stack([wl.q_rows(w, l) for l in range(L)])).to(device)
+    op = torch.empty((T, Hq, C, D), device=device)
+    lp = torch.empty((T, Hq, C), device=device)
+    out = torch.empty((L, T, Hq, D), device=device)
+    lse = torch.empty((L, T, Hq), device=device)
+
+    def step():
+        kvq.kvq_stream_decode(host, slots, q, Hq, T, n_kv, chunk, w.scale, op, lp, out, lse,
+                              compute=compute, copy=copy)
+
+    for _ in range(args.warmup):
+        step()
+    kvq.kvq_check(compute)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id(torch, device)) as clocks:
+        barrier(device)
+        torch.cuda.synchronize(device)
+        t0.record(compute)
+        for _ in range(args.steps):
+            step()
+        t1.record(compute)
+        torch.cuda.synchronize(device)
+        barrier(device)
+    kvq.kvq_check(compute)
+    ms = reduce_max(t0.elapsed_time(t1) / args.steps, device)
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    kv_bytes = L * n_kv * KV_BYTES_PER_TOKEN_LAYER(w)
+    peak = h2d_peak(torch, device, kv_bytes // L)
+    cl = clocks.summary()
+    res = None
+    if rank == 0:
+        gbs = world * kv_bytes / (ms * 1e-3) / 1e9
+        res = {
+            "metric": STREAM_METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "q8_0 K / q4_0 V x f16 q, f32 accumulate", "data": "synthetic",
+            "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": w.n_kv_heads,
+                       "head_dim": D, "context": n_kv, "query_tokens": T, "chunk": chunk,
+                       "seed": w.seed, "host_cache_bytes": kv_bytes, "slots": 2},
+            "query_tok_per_s": round(world * L * T / (ms * 1e-3), 2),
+            "roofline": {"bound": "h2d", "kernel": "kvq_stream_decode (copy stream)",
+                         "achieved": round(gbs / world, 2), "peak": round(peak, 2),
+                         "peak_kind": "measured pinned H2D, best of 5, one layer's bytes",
+                         "unit": "GB/s", "frac": round(gbs / world / peak, 4), "traffic": None},
+            "gpu_launches": 2 * L * args.steps,
+            "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
+                       "reasons": cl["reasons"], "samples": cl["samples"]},
+        }
+    del host, slots
+    if world > 1:
+        dist.destroy_process_group()
+    return res
+
+
 PREFILL_METRIC = "q8_0/q4_0 chunked prefill attn: TFLOP/s (% of tensor peak), query-tok/s at 262k ctx"
 
 
@@ -494,7 +596,7 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="verify262k",
-                    choices=["verify262k", "decode65k", "tiny", "prefill262k"])
+                    choices=["verify262k", "decode65k", "tiny", "prefill262k", "stream262k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="profile a smaller case of the same kernel: only this many layers")
@@ -509,6 +611,8 @@ def main(argv=None) -> int:
         res = run_reference(args, w)
     elif w.mode == "prefill":
         res = run_prefill(args, w)
+    elif w.mode == "stream":
+        res = run_stream(args, w)
     else:
         res = run_ours(args, w)
         if res is not None and world == 1 and not args.no_cpu_baseline:

@@ -72,7 +72,8 @@ constexpr float M_INIT = -1.0e30f;
 constexpr uint32_t COL_O = 0, COL_Q = 256, COL_S0 = 384;  // S buffer b at COL_S0 + BN b
 
 struct PfSmemHead {
-    uint64_t raw_full[2], raw_free[2], kv_full[2], s_full[2], p_full[2], pv_done[2], q_ready;
+    uint64_t raw_full[2], raw_free[2], k_full[2], v_full[2], s_full[2], p_full[2], pv_done[2],
+        q_ready;
     uint32_t tmem_base;
     int abort;
 };
@@ -151,7 +152,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&hd.raw_full[i], 1);
             ptx::mbar_init(&hd.raw_free[i], N_DEQ);
-            ptx::mbar_init(&hd.kv_full[i], N_DEQ);
+            ptx::mbar_init(&hd.k_full[i], N_DEQ);
+            ptx::mbar_init(&hd.v_full[i], N_DEQ);
             ptx::mbar_init(&hd.s_full[i], 1);
             ptx::mbar_init(&hd.p_full[i], N_SOFT);
             ptx::mbar_init(&hd.pv_done[i], 1);
@@ -323,13 +325,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         }
     } else if (warp < W_PROD) {
         // ================================================================ dequant
+        // unit u of a tile = (key r, block bk); a warp takes 8 keys x 4 blocks so
+        // that the 8 lanes of each quarter-warp store 8 different keys of one
+        // block: with the swizzle those land in 8 different bank groups
         const int dt = threadIdx.x - N_SOFT * 32;  // 0..255
         for (int j = 0; j < ntiles; ++j) {
             const int b = j & 1;
+            // K^ of tile j overwrites buffer b once QK^T of tile j-2 is done (s_full);
+            // V^ once PV of tile j-2 is done (pv_done)
             bool ok = true;
             if (lane == 0)
                 ok = ptx::mbar_wait_bounded(&hd.raw_full[b], (j >> 1) & 1, abort, WAIT_NS) &&
-                     ptx::mbar_wait_bounded(&hd.pv_done[b], ((j >> 1) & 1) ^ 1, abort, WAIT_NS);
+                     ptx::mbar_wait_bounded(&hd.s_full[b], ((j >> 1) & 1) ^ 1, abort, WAIT_NS);
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
                 if (lane == 0)
                     fail();
@@ -343,11 +350,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
             uint8_t *vh = smem + OFF_VH + b * TILE_H;
 #pragma unroll 1
             for (int u = dt; u < BN * 8; u += N_DEQ * 32) {
-                const int r = u >> 3, bk = u & 7;
-                uint32_t w[8];
+                const int grp = u >> 5, ln = u & 31;
+                const int r = (grp % (BN / 8)) * 8 + (ln & 7), bk = (grp / (BN / 8)) * 4 + (ln >> 3);
                 if (r < rows) {
                     // ---- K block: d (fp16) + 32 int8
                     const uint8_t *src = rk + r * KROW + 34 * bk;
+                    uint32_t w[8];
                     uint32_t d16;
                     if ((bk & 1) == 0) {  // block starts 4-byte aligned: d, q0, q1 | ...
                         uint32_t x[9];
@@ -373,9 +381,34 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
                         sts128(kh + sw_off(r, 32 * bk + 8 * m4), x0[0], x0[1], x1[0], x1[1]);
                         sts128(kl + sw_off(r, 32 * bk + 8 * m4), r0[0], r0[1], r1[0], r1[1]);
                     }
+                } else {
+#pragma unroll
+                    for (int m4 = 0; m4 < 4; ++m4) {
+                        sts128(kh + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
+                        sts128(kl + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
+                    }
+                }
+            }
+            ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+            __syncwarp();
+            if (lane == 0)
+                ptx::mbar_arrive(&hd.k_full[b]);
+            if (lane == 0)
+                ok = ptx::mbar_wait_bounded(&hd.pv_done[b], ((j >> 1) & 1) ^ 1, abort, WAIT_NS);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                if (lane == 0)
+                    fail();
+                break;
+            }
+#pragma unroll 1
+            for (int u = dt; u < BN * 8; u += N_DEQ * 32) {
+                const int grp = u >> 5, ln = u & 31;
+                const int r = (grp % (BN / 8)) * 8 + (ln & 7), bk = (grp / (BN / 8)) * 4 + (ln >> 3);
+                if (r < rows) {
                     // ---- V block: d (fp16) + 16 bytes of nibbles
                     const uint8_t *vsrc = rv + r * VROW + 18 * bk;
                     uint32_t vw[4];
+                    uint32_t d16;
                     if ((bk & 1) == 0) {
                         uint32_t x[5];
 #pragma unroll
@@ -396,7 +429,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
                     uint32_t lo[8], hi[8];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        v2(ptx::prmt(vw[i], 0u, 0x4140), dv, lo[2 * i], hi[2 * i]);      // bytes 0, 1
+                        v2(ptx::prmt(vw[i], 0u, 0x4140), dv, lo[2 * i], hi[2 * i]);          // bytes 0, 1
                         v2(ptx::prmt(vw[i], 0u, 0x4342), dv, lo[2 * i + 1], hi[2 * i + 1]);  // bytes 2, 3
                     }
                     sts128(vh + sw_off(r, 32 * bk + 0), lo[0], lo[1], lo[2], lo[3]);
@@ -404,20 +437,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
                     sts128(vh + sw_off(r, 32 * bk + 16), hi[0], hi[1], hi[2], hi[3]);
                     sts128(vh + sw_off(r, 32 * bk + 24), hi[4], hi[5], hi[6], hi[7]);
                 } else {
-                    // keys past the end: zero K and V so that 0-weight products stay 0
+                    // keys past the end: zero V so that 0-weight products stay 0
 #pragma unroll
-                    for (int m4 = 0; m4 < 4; ++m4) {
-                        sts128(kh + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
-                        sts128(kl + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
+                    for (int m4 = 0; m4 < 4; ++m4)
                         sts128(vh + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
-                    }
                 }
             }
-            ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+            ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(&hd.raw_free[b]);
-                ptx::mbar_arrive(&hd.kv_full[b]);
+                ptx::mbar_arrive(&hd.v_full[b]);
             }
         }
     } else if (warp == W_PROD) {
@@ -454,7 +484,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
             bool ok = ptx::mbar_wait_bounded(&hd.q_ready, 0, abort, WAIT_NS);
             auto issue_pv = [&](int jj) -> bool {
                 const int bb = jj & 1;
-                if (!ptx::mbar_wait_bounded(&hd.p_full[bb], (jj >> 1) & 1, abort, WAIT_NS))
+                if (!ptx::mbar_wait_bounded(&hd.v_full[bb], (jj >> 1) & 1, abort, WAIT_NS) ||
+                    !ptx::mbar_wait_bounded(&hd.p_full[bb], (jj >> 1) & 1, abort, WAIT_NS))
                     return false;
                 ptx::tc_fence_after();
                 const uint8_t *vh = smem + OFF_VH + bb * TILE_H;
@@ -469,7 +500,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
             };
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int b = j & 1;
-                ok = ptx::mbar_wait_bounded(&hd.kv_full[b], (j >> 1) & 1, abort, WAIT_NS) &&
+                ok = ptx::mbar_wait_bounded(&hd.k_full[b], (j >> 1) & 1, abort, WAIT_NS) &&
                      (j < 2 || ptx::mbar_wait_bounded(&hd.pv_done[b], ((j >> 1) - 1) & 1, abort,
                                                        WAIT_NS));
                 if (!ok)

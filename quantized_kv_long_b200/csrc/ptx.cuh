@@ -64,24 +64,37 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep inside the
+// instruction (up to `hint_ns`) until the phase completes, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase of `bar` with the given parity to complete.
-// Gives up (returns false) after `limit_ns` of wall time, or at once when
-// *abort is set by another thread of the CTA.
+// Gives up (returns false) after `limit_ns` of wall time, or once *abort is
+// set by another thread of the CTA (checked between sleeps of <= 0.1 ms).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort, uint64_t limit_ns)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity))
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u))
             return true;
-        if ((it & 63u) == 0) {
-            if (*abort)
-                return false;
-            if (globaltimer_ns() - t0 > limit_ns)
-                return false;
-        }
+        if (*abort)
+            return false;
+        if (globaltimer_ns() - t0 > limit_ns)
+            return false;
     }
 }
 
