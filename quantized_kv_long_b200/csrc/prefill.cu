@@ -13,23 +13,28 @@
 //  * prefill_tc_kernel -- the tensor-core path (tcgen05, TMEM) for rows that
 //    see at least PF_MIN_KEYS keys.  One CTA per (128 query rows of one KV
 //    head's group, KV head, layer); rows are (token, q head) pairs.  Per tile
-//    of 48 keys:
-//      - a producer warp bulk-copies the tile's raw Q8_0 K head-rows (48 x
-//        272 B) and Q4_0 V head-rows (48 x 144 B) into a 2-deep staging ring;
-//      - 8 dequant warps turn them into f16 tiles in shared memory with
-//        128-byte swizzle: K^ = d * q as an exact two-part f16 sum (K^hi =
-//        RN_f16(d q), K^lo = fma(d, q, -K^hi)), K-major (keys x head_dim), and
+//    of 32 keys:
+//      - a producer thread bulk-copies the tile's raw Q8_0 K head-rows (32 x
+//        272 B) and Q4_0 V head-rows (32 x 144 B) into a 4-slot staging ring,
+//        so that three tiles of copies are in flight while one is dequantized;
+//      - 8 dequant warps (one (key, block) unit of K and one of V per thread)
+//        turn them into f16 tiles in shared memory with 128-byte swizzle:
+//        K^ = d * q as an exact two-part f16 sum (K^hi = RN_f16(d q),
+//        K^lo = fma(d, q, -K^hi)), K-major (keys x head_dim), and
 //        V^ = RN_f16(d * (u - 8)) MN-major (keys x head_dim), zeros past the
-//        end;
-//      - one thread issues tcgen05.mma: S = Q K^hi^T + Q K^lo^T (A = Q held
-//        in tensor memory, M = 128, N = 48, K = 256, twice) into a double-
-//        buffered S in TMEM -- exact products, so the logits carry only fp32
-//        rounding -- then O += P V^ (A = P in TMEM, written over S; N = 256,
-//        K = 48) into the fp32 O accumulator in TMEM (256 columns);
+//        end; two slots of each;
+//      - the MMA warp (warp-converged; one elected lane issues) runs
+//        tcgen05.mma: S = Q K^hi^T + Q K^lo^T (A = Q held in tensor memory,
+//        M = 128, N = 32, K = 256, twice) into one of 4 S slots in TMEM --
+//        exact products, so the logits carry only fp32 rounding -- then
+//        O += P V^ (A = P in TMEM, written over its S slot; N = 256, K = 32)
+//        into the fp32 O accumulator in TMEM (256 columns).  A slot is
+//        rewritten four tiles later, once that tile's PV has finished, so the
+//        tensor pipe never waits for its own last PV;
 //      - 4 softmax warps own one query row per thread (its TMEM lane): they
 //        read S, apply the causal mask, keep a lazy running max (moves only
 //        when a score exceeds it by 8 in log2 units, with an exact rescale of
-//        O in TMEM) and write P = 2^(s - m) as f16 back into TMEM.
+//        O in TMEM) and write P = 2^(s - m) as f16 back into the slot.
 //    V^ and P carry one f16 rounding each (relative 2^-11).  These errors are
 //    independent per key and average over the visible keys, but a row whose
 //    softmax is peaked (a large query component on an x8 outlier channel) can
@@ -56,10 +61,14 @@ namespace kvq {
 namespace {
 
 constexpr int PF_MIN_KEYS = 16384;
-constexpr int BM = 128, BN = 48, HD = 256;
+constexpr int BM = 128, BN = 32, HD = 256;
 constexpr int KROW = 272, VROW = 144;
-constexpr int RAW_K = BN * KROW, RAW_V = BN * VROW, RAW_BYTES = RAW_K + RAW_V;
-constexpr int TILE_H = BN * HD * 2;  // one f16 tile of 48 keys x 256 dims: 24 KB
+constexpr int RAW_K = BN * KROW, RAW_V = BN * VROW, RAW_BYTES = RAW_K + RAW_V;  // 13,312 B
+constexpr int TILE_H = BN * HD * 2;  // one f16 tile of 32 keys x 256 dims: 16 KB
+constexpr int NR = 4;  // raw staging slots (bulk copies in flight ahead of the dequant)
+constexpr int NB = 2;  // f16 K^hi / K^lo / V^ tile slots
+constexpr int NS = 4;  // S / P slots in tensor memory
+constexpr int LA = 1;  // the PV of tile j - LA is issued after the QK^T of tile j
 constexpr int N_SOFT = 4, N_DEQ = 8;
 constexpr int W_PROD = N_SOFT + N_DEQ, W_MMA = W_PROD + 1;
 constexpr int PF_THREADS = (W_MMA + 1) * 32;  // 14 warps
@@ -68,19 +77,29 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float TAU = 8.0f;
 constexpr float M_INIT = -1.0e30f;
-// tensor-memory columns
-constexpr uint32_t COL_O = 0, COL_Q = 256, COL_S0 = 384;  // S buffer b at COL_S0 + BN b
+// tensor-memory columns: O (fp32, 256), Q (f16 pairs, 128), S slot s at COL_S0 + BN s
+// (P of that tile, f16 pairs, is written over the first BN / 2 columns of its slot)
+constexpr uint32_t COL_O = 0, COL_Q = 256, COL_S0 = 384;
+static_assert(COL_S0 + NS * BN <= 512, "tensor-memory columns");
+static_assert(BN * 8 == N_DEQ * 32, "one K unit and one V unit per dequant thread and tile");
+static_assert(NB <= NS, "a K^ slot is reused only after the QK^T that read it");
 
 struct PfSmemHead {
-    uint64_t raw_full[2], raw_free[2], k_full[2], v_full[2], s_full[2], p_full[2], pv_done[2],
-        q_ready;
+    uint64_t raw_full[NR], raw_free[NR], k_full[NB], v_full[NB], s_full[NS], p_full[NS],
+        pv_done[NS], q_ready;
     uint32_t tmem_base;
     int abort;
 };
-// layout: [K^hi 2 x 24K][K^lo 2 x 24K][V^ 2 x 24K][raw 2 x 19,968][head], base 1024-aligned
-constexpr int OFF_KH = 0, OFF_KL = 2 * TILE_H, OFF_VH = 4 * TILE_H, OFF_RAW = 6 * TILE_H;
-constexpr int OFF_HEAD = OFF_RAW + 2 * RAW_BYTES;
+// layout: [K^hi NB x 16K][K^lo NB x 16K][V^ NB x 16K][raw NR x 13,312][head], base 1024-aligned
+constexpr int OFF_KH = 0, OFF_KL = NB * TILE_H, OFF_VH = 2 * NB * TILE_H;
+constexpr int OFF_RAW = 3 * NB * TILE_H;
+constexpr int OFF_HEAD = OFF_RAW + NR * RAW_BYTES;
 constexpr int PF_SMEM = OFF_HEAD + (int)sizeof(PfSmemHead) + 1024;  // + alignment slack
+static_assert(PF_SMEM <= 232448, "dynamic shared memory per block");
+
+// slot and phase parity of tile t in a ring of S slots
+__device__ __forceinline__ int slot(int t, int S) { return t % S; }
+__device__ __forceinline__ uint32_t par(int t, int S) { return (uint32_t)(t / S) & 1u; }
 
 // byte offset of (row, dim) in a [BN rows x 256 dims] f16 tile stored as four
 // 1024-aligned column blocks of [BN rows x 128 B] with the 128-byte swizzle
@@ -149,11 +168,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
     volatile int *abort = &hd.abort;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NR; ++i) {
             ptx::mbar_init(&hd.raw_full[i], 1);
             ptx::mbar_init(&hd.raw_free[i], N_DEQ);
+        }
+        for (int i = 0; i < NB; ++i) {
             ptx::mbar_init(&hd.k_full[i], N_DEQ);
             ptx::mbar_init(&hd.v_full[i], N_DEQ);
+        }
+        for (int i = 0; i < NS; ++i) {
             ptx::mbar_init(&hd.s_full[i], 1);
             ptx::mbar_init(&hd.p_full[i], N_SOFT);
             ptx::mbar_init(&hd.pv_done[i], 1);
@@ -175,6 +198,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
             *abort = 1;
             report_timeout(a.status);
         }
+    };
+    // warp-wide bounded wait: lane 0 waits, the result is broadcast
+    auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+        bool ok = true;
+        if (lane == 0)
+            ok = ptx::mbar_wait_bounded(bar, parity, abort, WAIT_NS);
+        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     };
 
     if (warp < N_SOFT) {
@@ -210,12 +240,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         const float sl2 = a.scale * LOG2E;
         float m = M_INIT, l = 0.0f;
         for (int j = 0; j < ntiles; ++j) {
-            const int b = j & 1;
-            const uint32_t scol = COL_S0 + BN * b;
-            bool ok = true;
-            if (lane == 0)
-                ok = ptx::mbar_wait_bounded(&hd.s_full[b], (j >> 1) & 1, abort, WAIT_NS);
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+            const int sb = slot(j, NS);
+            const uint32_t scol = COL_S0 + BN * sb;
+            if (!wwait(&hd.s_full[sb], par(j, NS))) {
                 if (lane == 0)
                     fail();
                 break;
@@ -238,23 +265,26 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
                     if (kj0 + e > lim)
                         s[e] = -INFINITY;
             }
-            float mx = s[0];
+            // tree reduction (independent chains) for the tile max
+            float mx8[8];
 #pragma unroll
-            for (int e = 1; e < BN; ++e)
-                mx = fmaxf(mx, s[e]);
+            for (int e = 0; e < 8; ++e)
+                mx8[e] = s[e];
+#pragma unroll
+            for (int e = 8; e < BN; ++e)
+                mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             float alpha = 1.0f;
             if (mx > m + TAU) {
                 alpha = ptx::ex2(m - mx);
                 m = mx;
                 l *= alpha;
             }
-            // rescale O (rare): the whole warp takes part once any lane needs it
+            // rescale O (rare): the whole warp takes part once any lane needs it, after
+            // the PV of the previous tile has finished
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-                bool okp = true;
-                if (lane == 0)
-                    okp = ptx::mbar_wait_bounded(&hd.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1,
-                                                 abort, WAIT_NS);
-                if (!__shfl_sync(0xffffffffu, okp ? 1 : 0, 0)) {
+                if (!wwait(&hd.pv_done[slot(j - 1, NS)], par(j - 1, NS))) {
                     if (lane == 0)
                         fail();
                     break;
@@ -271,34 +301,29 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
                 }
                 ptx::tmem_wait_st();
             }
-            // P = 2^(s - m) in f16 over the first BN/2 columns of this S buffer
-            uint32_t pk[BN / 2 + 8];
+            // P = 2^(s - m) in f16 (keys 2e, 2e + 1 in column e) over the first BN / 2
+            // columns of this S slot
+            uint32_t pk[BN / 2];
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < BN / 2; ++e) {
                 const float p0 = ptx::ex2(s[2 * e] - m), p1 = ptx::ex2(s[2 * e + 1] - m);
-                l += p0 + p1;
+                ls[e & 3] += p0 + p1;
                 pk[e] = ptx::h2_bits(__floats2half2_rn(p0, p1));
             }
-            ptx::tmem_st16(lane_addr + scol, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-            // the last 8 P columns (keys 32..47); the 8 columns after them belong to
-            // this S buffer too and are rewritten by the next QK^T
-#pragma unroll
-            for (int e = BN / 2; e < BN / 2 + 8; ++e)
-                pk[e] = 0u;
-            ptx::tmem_st16(lane_addr + scol + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            static_assert(BN / 2 == 16, "P of one tile is one 16-column TMEM store");
+            ptx::tmem_st16(lane_addr + scol, pk);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                ptx::mbar_arrive(&hd.p_full[b]);
+                ptx::mbar_arrive(&hd.p_full[sb]);
         }
         // ---- epilogue: out = O / l, lse = (m + log2 l) ln 2
         if (!*abort) {
             const int last = ntiles - 1;
-            bool ok = true;
-            if (lane == 0)
-                ok = ptx::mbar_wait_bounded(&hd.pv_done[last & 1], (last >> 1) & 1, abort, WAIT_NS);
-            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+            if (wwait(&hd.pv_done[slot(last, NS)], par(last, NS))) {
                 ptx::tc_fence_after();
                 const float inv = l > 0.0f ? 1.0f / l : 0.0f;
                 float4 *op = reinterpret_cast<float4 *>(
@@ -325,129 +350,123 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         }
     } else if (warp < W_PROD) {
         // ================================================================ dequant
-        // unit u of a tile = (key r, block bk); a warp takes 8 keys x 4 blocks so
-        // that the 8 lanes of each quarter-warp store 8 different keys of one
-        // block: with the swizzle those land in 8 different bank groups
+        // Each of the 256 dequant threads owns one (key r, block bk) unit of every
+        // tile, for K and for V.  A warp takes 8 keys x 4 blocks of one parity
+        // (bk = p, p+2, p+4, p+6): the even/odd alignment branch is uniform across
+        // the warp, the 8 lanes of each quarter-warp store 8 different keys of one
+        // block (8 different bank groups after the swizzle), and the raw 32-bit
+        // loads (rows 68 words apart, blocks 17 words apart) hit 32 different banks.
         const int dt = threadIdx.x - N_SOFT * 32;  // 0..255
+        const int grp = dt >> 5, ln = dt & 31;
+        const int r = (grp % (BN / 8)) * 8 + (ln & 7), bk = grp / (BN / 8) + 2 * (ln >> 3);
+        uint32_t off[4];  // swizzled offsets of dims 32 bk + 8 m4 of key r in an f16 tile
+#pragma unroll
+        for (int m4 = 0; m4 < 4; ++m4)
+            off[m4] = sw_off(r, 32 * bk + 8 * m4);
         for (int j = 0; j < ntiles; ++j) {
-            const int b = j & 1;
-            // K^ of tile j overwrites buffer b once QK^T of tile j-2 is done (s_full);
-            // V^ once PV of tile j-2 is done (pv_done)
-            bool ok = true;
-            if (lane == 0)
-                ok = ptx::mbar_wait_bounded(&hd.raw_full[b], (j >> 1) & 1, abort, WAIT_NS) &&
-                     ptx::mbar_wait_bounded(&hd.s_full[b], ((j >> 1) & 1) ^ 1, abort, WAIT_NS);
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+            const int rb = slot(j, NR), kb = slot(j, NB);
+            // raw tile j has landed; K^ slot kb is free once the QK^T of tile j - NB is done
+            if (!wwait(&hd.raw_full[rb], par(j, NR)) ||
+                (j >= NB && !wwait(&hd.s_full[slot(j - NB, NS)], par(j - NB, NS)))) {
                 if (lane == 0)
                     fail();
                 break;
             }
-            const int rows = (int)min((int64_t)BN, n_keys - (int64_t)j * BN);
-            const uint8_t *rk = smem + OFF_RAW + b * RAW_BYTES;
+            const bool in = r < (int)min((int64_t)BN, n_keys - (int64_t)j * BN);
+            const uint8_t *rk = smem + OFF_RAW + rb * RAW_BYTES;
             const uint8_t *rv = rk + RAW_K;
-            uint8_t *kh = smem + OFF_KH + b * TILE_H;
-            uint8_t *kl = smem + OFF_KL + b * TILE_H;
-            uint8_t *vh = smem + OFF_VH + b * TILE_H;
-#pragma unroll 1
-            for (int u = dt; u < BN * 8; u += N_DEQ * 32) {
-                const int grp = u >> 5, ln = u & 31;
-                const int r = (grp % (BN / 8)) * 8 + (ln & 7), bk = (grp / (BN / 8)) * 4 + (ln >> 3);
-                if (r < rows) {
-                    // ---- K block: d (fp16) + 32 int8
-                    const uint8_t *src = rk + r * KROW + 34 * bk;
-                    uint32_t w[8];
-                    uint32_t d16;
-                    if ((bk & 1) == 0) {  // block starts 4-byte aligned: d, q0, q1 | ...
-                        uint32_t x[9];
+            uint8_t *kh = smem + OFF_KH + kb * TILE_H;
+            uint8_t *kl = smem + OFF_KL + kb * TILE_H;
+            uint8_t *vh = smem + OFF_VH + kb * TILE_H;
+            if (in) {
+                // ---- K block: d (fp16) + 32 int8
+                const uint8_t *src = rk + r * KROW + 34 * bk;
+                uint32_t w[8];
+                uint32_t d16;
+                if ((bk & 1) == 0) {  // block starts 4-byte aligned: d, q0, q1 | ...
+                    uint32_t x[9];
 #pragma unroll
-                        for (int i = 0; i < 9; ++i)
-                            x[i] = lds32(src + 4 * i);
-                        d16 = x[0] & 0xFFFFu;
+                    for (int q = 0; q < 9; ++q)
+                        x[q] = lds32(src + 4 * q);
+                    d16 = x[0] & 0xFFFFu;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            w[i] = ptx::prmt(x[i], x[i + 1], 0x5432);
-                    } else {              // qs start 4-byte aligned
-                        d16 = lds16(src);
+                    for (int q = 0; q < 8; ++q)
+                        w[q] = ptx::prmt(x[q], x[q + 1], 0x5432);
+                } else {              // qs start 4-byte aligned
+                    d16 = lds16(src);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            w[i] = lds32(src + 2 + 4 * i);
-                    }
-                    const __half2 d2 = dup_h(d16);
+                    for (int q = 0; q < 8; ++q)
+                        w[q] = lds32(src + 2 + 4 * q);
+                }
+                const __half2 d2 = dup_h(d16);
 #pragma unroll
-                    for (int m4 = 0; m4 < 4; ++m4) {
-                        uint32_t x0[2], x1[2], r0[2], r1[2];
-                        k4(w[2 * m4], d2, x0, r0);
-                        k4(w[2 * m4 + 1], d2, x1, r1);
-                        sts128(kh + sw_off(r, 32 * bk + 8 * m4), x0[0], x0[1], x1[0], x1[1]);
-                        sts128(kl + sw_off(r, 32 * bk + 8 * m4), r0[0], r0[1], r1[0], r1[1]);
-                    }
-                } else {
+                for (int m4 = 0; m4 < 4; ++m4) {
+                    uint32_t x0[2], x1[2], r0[2], r1[2];
+                    k4(w[2 * m4], d2, x0, r0);
+                    k4(w[2 * m4 + 1], d2, x1, r1);
+                    sts128(kh + off[m4], x0[0], x0[1], x1[0], x1[1]);
+                    sts128(kl + off[m4], r0[0], r0[1], r1[0], r1[1]);
+                }
+            } else {
 #pragma unroll
-                    for (int m4 = 0; m4 < 4; ++m4) {
-                        sts128(kh + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
-                        sts128(kl + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
-                    }
+                for (int m4 = 0; m4 < 4; ++m4) {
+                    sts128(kh + off[m4], 0u, 0u, 0u, 0u);
+                    sts128(kl + off[m4], 0u, 0u, 0u, 0u);
                 }
             }
             ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
             __syncwarp();
             if (lane == 0)
-                ptx::mbar_arrive(&hd.k_full[b]);
-            if (lane == 0)
-                ok = ptx::mbar_wait_bounded(&hd.pv_done[b], ((j >> 1) & 1) ^ 1, abort, WAIT_NS);
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                ptx::mbar_arrive(&hd.k_full[kb]);
+            // V^ slot kb is free once the PV of tile j - NB is done
+            if (j >= NB && !wwait(&hd.pv_done[slot(j - NB, NS)], par(j - NB, NS))) {
                 if (lane == 0)
                     fail();
                 break;
             }
-#pragma unroll 1
-            for (int u = dt; u < BN * 8; u += N_DEQ * 32) {
-                const int grp = u >> 5, ln = u & 31;
-                const int r = (grp % (BN / 8)) * 8 + (ln & 7), bk = (grp / (BN / 8)) * 4 + (ln >> 3);
-                if (r < rows) {
-                    // ---- V block: d (fp16) + 16 bytes of nibbles
-                    const uint8_t *vsrc = rv + r * VROW + 18 * bk;
-                    uint32_t vw[4];
-                    uint32_t d16;
-                    if ((bk & 1) == 0) {
-                        uint32_t x[5];
+            if (in) {
+                // ---- V block: d (fp16) + 16 bytes of nibbles
+                const uint8_t *vsrc = rv + r * VROW + 18 * bk;
+                uint32_t vw[4];
+                uint32_t d16;
+                if ((bk & 1) == 0) {
+                    uint32_t x[5];
 #pragma unroll
-                        for (int i = 0; i < 5; ++i)
-                            x[i] = lds32(vsrc + 4 * i);
-                        d16 = x[0] & 0xFFFFu;
+                    for (int q = 0; q < 5; ++q)
+                        x[q] = lds32(vsrc + 4 * q);
+                    d16 = x[0] & 0xFFFFu;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            vw[i] = ptx::prmt(x[i], x[i + 1], 0x5432);
-                    } else {
-                        d16 = lds16(vsrc);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            vw[i] = lds32(vsrc + 2 + 4 * i);
-                    }
-                    const __half2 dv = dup_h(d16);
-                    // byte j of the block: element j (low nibble), element j + 16 (high)
-                    uint32_t lo[8], hi[8];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        v2(ptx::prmt(vw[i], 0u, 0x4140), dv, lo[2 * i], hi[2 * i]);          // bytes 0, 1
-                        v2(ptx::prmt(vw[i], 0u, 0x4342), dv, lo[2 * i + 1], hi[2 * i + 1]);  // bytes 2, 3
-                    }
-                    sts128(vh + sw_off(r, 32 * bk + 0), lo[0], lo[1], lo[2], lo[3]);
-                    sts128(vh + sw_off(r, 32 * bk + 8), lo[4], lo[5], lo[6], lo[7]);
-                    sts128(vh + sw_off(r, 32 * bk + 16), hi[0], hi[1], hi[2], hi[3]);
-                    sts128(vh + sw_off(r, 32 * bk + 24), hi[4], hi[5], hi[6], hi[7]);
+                    for (int q = 0; q < 4; ++q)
+                        vw[q] = ptx::prmt(x[q], x[q + 1], 0x5432);
                 } else {
-                    // keys past the end: zero V so that 0-weight products stay 0
+                    d16 = lds16(vsrc);
 #pragma unroll
-                    for (int m4 = 0; m4 < 4; ++m4)
-                        sts128(vh + sw_off(r, 32 * bk + 8 * m4), 0u, 0u, 0u, 0u);
+                    for (int q = 0; q < 4; ++q)
+                        vw[q] = lds32(vsrc + 2 + 4 * q);
                 }
+                const __half2 dv = dup_h(d16);
+                // byte j of the block: element j (low nibble), element j + 16 (high)
+                uint32_t lo[8], hi[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    v2(ptx::prmt(vw[q], 0u, 0x4140), dv, lo[2 * q], hi[2 * q]);          // bytes 0, 1
+                    v2(ptx::prmt(vw[q], 0u, 0x4342), dv, lo[2 * q + 1], hi[2 * q + 1]);  // bytes 2, 3
+                }
+                sts128(vh + off[0], lo[0], lo[1], lo[2], lo[3]);
+                sts128(vh + off[1], lo[4], lo[5], lo[6], lo[7]);
+                sts128(vh + off[2], hi[0], hi[1], hi[2], hi[3]);
+                sts128(vh + off[3], hi[4], hi[5], hi[6], hi[7]);
+            } else {
+                // keys past the end: zero V so that 0-weight products stay 0
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4)
+                    sts128(vh + off[m4], 0u, 0u, 0u, 0u);
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                ptx::mbar_arrive(&hd.raw_free[b]);
-                ptx::mbar_arrive(&hd.v_full[b]);
+                ptx::mbar_arrive(&hd.raw_free[rb]);
+                ptx::mbar_arrive(&hd.v_full[kb]);
             }
         }
     } else if (warp == W_PROD) {
@@ -455,83 +474,96 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         if (lane == 0) {
             int issued = 0;
             for (int j = 0; j < ntiles; ++j) {
-                const int b = j & 1;
-                if (*abort ||
-                    !ptx::mbar_wait_bounded(&hd.raw_free[b], ((j >> 1) & 1) ^ 1, abort, WAIT_NS) ||
-                    (j >= 2 && !ptx::mbar_wait_bounded(&hd.raw_full[b], ((j >> 1) - 1) & 1, abort,
-                                                       WAIT_NS))) {
+                const int rb = slot(j, NR);
+                // raw slot rb is free once every dequant warp is done with tile j - NR
+                if (*abort || (j >= NR && !ptx::mbar_wait_bounded(&hd.raw_free[rb], par(j - NR, NR),
+                                                                   abort, WAIT_NS))) {
                     fail();
                     break;
                 }
                 const int rows = (int)min((int64_t)BN, n_keys - (int64_t)j * BN);
-                uint8_t *dst = smem + OFF_RAW + b * RAW_BYTES;
-                ptx::mbar_arrive_expect_tx(&hd.raw_full[b], rows * (KROW + VROW));
-                ptx::bulk_g2s(dst, kg + (int64_t)j * RAW_K, rows * KROW, &hd.raw_full[b]);
-                ptx::bulk_g2s(dst + RAW_K, vg + (int64_t)j * RAW_V, rows * VROW, &hd.raw_full[b]);
+                uint8_t *dst = smem + OFF_RAW + rb * RAW_BYTES;
+                ptx::mbar_arrive_expect_tx(&hd.raw_full[rb], rows * (KROW + VROW));
+                ptx::bulk_g2s(dst, kg + (int64_t)j * RAW_K, rows * KROW, &hd.raw_full[rb]);
+                ptx::bulk_g2s(dst + RAW_K, vg + (int64_t)j * RAW_V, rows * VROW, &hd.raw_full[rb]);
                 issued = j + 1;
             }
+            // no copy may still be landing when the CTA exits
             int none = 0;
-            for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-                if (!ptx::mbar_wait_bounded(&hd.raw_full[j & 1], (j >> 1) & 1, &none, WAIT_NS))
+            for (int j = (issued > NR ? issued - NR : 0); j < issued; ++j)
+                if (!ptx::mbar_wait_bounded(&hd.raw_full[slot(j, NR)], par(j, NR), &none, WAIT_NS))
                     report_timeout(a.status);
         }
     } else {
         // ================================================================ MMA issue
-        if (lane == 0) {
-            const uint32_t id_qk = ptx::idesc_f16_f32(BM, BN, false, false);
-            const uint32_t id_pv = ptx::idesc_f16_f32(BM, HD, false, true);
-            int committed = -1;  // last tile whose PV was committed
-            bool ok = ptx::mbar_wait_bounded(&hd.q_ready, 0, abort, WAIT_NS);
-            auto issue_pv = [&](int jj) -> bool {
-                const int bb = jj & 1;
-                if (!ptx::mbar_wait_bounded(&hd.v_full[bb], (jj >> 1) & 1, abort, WAIT_NS) ||
-                    !ptx::mbar_wait_bounded(&hd.p_full[bb], (jj >> 1) & 1, abort, WAIT_NS))
-                    return false;
-                ptx::tc_fence_after();
-                const uint8_t *vh = smem + OFF_VH + bb * TILE_H;
+        // The whole warp runs this loop (descriptors stay warp-uniform); the
+        // elected lane issues every MMA and commit, so all tcgen05 work of the
+        // CTA comes from one thread and each commit covers what came before.
+        const uint32_t leader = ptx::elect_one();
+        const uint32_t id_qk = ptx::idesc_f16_f32(BM, BN, false, false);
+        const uint32_t id_pv = ptx::idesc_f16_f32(BM, HD, false, true);
+        // descriptors of slot 0; slots and k-steps add to the start-address field
+        // (16-byte units; every tile lies inside one 256 KB window)
+        const uint64_t dk_hi0 = ptx::smem_desc_sw128(smem + OFF_KH, 16, 1024);
+        const uint64_t dk_lo0 = ptx::smem_desc_sw128(smem + OFF_KL, 16, 1024);
+        const uint64_t dv0 = ptx::smem_desc_sw128(smem + OFF_VH, BN * 128, 1024);
+        int committed = -1;  // last tile whose PV was committed
+        bool ok = wwait(&hd.q_ready, 0);
+        auto issue_pv = [&](int jj) -> bool {
+            const int vb = slot(jj, NB), sb = slot(jj, NS);
+            if (!wwait(&hd.v_full[vb], par(jj, NB)) || !wwait(&hd.p_full[sb], par(jj, NS)))
+                return false;
+            ptx::tc_fence_after();
+            if (leader) {
+                const uint64_t dv = dv0 + (uint64_t)((vb * TILE_H) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    ptx::umma_f16_ts(tbase + COL_O, tbase + COL_S0 + BN * bb + 8 * kk,
-                                     ptx::smem_desc_sw128(vh + kk * 2 * 1024, BN * 128, 1024), id_pv,
-                                     jj > 0 || kk > 0);
-                ptx::umma_commit(&hd.pv_done[bb]);
-                committed = jj;
-                return true;
-            };
-            for (int j = 0; ok && j < ntiles; ++j) {
-                const int b = j & 1;
-                ok = ptx::mbar_wait_bounded(&hd.k_full[b], (j >> 1) & 1, abort, WAIT_NS) &&
-                     (j < 2 || ptx::mbar_wait_bounded(&hd.pv_done[b], ((j >> 1) - 1) & 1, abort,
-                                                       WAIT_NS));
-                if (!ok)
-                    break;
-                ptx::tc_fence_after();
+                    ptx::umma_f16_ts(tbase + COL_O, tbase + COL_S0 + BN * sb + 8 * kk,
+                                     dv + (uint64_t)((kk * 2 * 1024) >> 4), id_pv, jj > 0 || kk > 0);
+                ptx::umma_commit(&hd.pv_done[sb]);
+            }
+            __syncwarp();
+            committed = jj;
+            return true;
+        };
+        for (int j = 0; ok && j < ntiles; ++j) {
+            const int kb = slot(j, NB), sb = slot(j, NS);
+            // K^ of tile j is ready; S slot sb (P of tile j - NS) is free once that PV is done
+            ok = wwait(&hd.k_full[kb], par(j, NB)) &&
+                 (j < NS || wwait(&hd.pv_done[sb], par(j - NS, NS)));
+            if (!ok)
+                break;
+            ptx::tc_fence_after();
+            if (leader) {
                 // S = Q K^hi^T + Q K^lo^T: exact products of q and d*q_int, fp32 sums
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
-                    const uint8_t *kt = smem + (part ? OFF_KL : OFF_KH) + b * TILE_H;
+                    const uint64_t dk = (part ? dk_lo0 : dk_hi0) + (uint64_t)((kb * TILE_H) >> 4);
 #pragma unroll
                     for (int ks = 0; ks < HD / 16; ++ks)
-                        ptx::umma_f16_ts(tbase + COL_S0 + BN * b, tbase + COL_Q + 8 * ks,
-                                         ptx::smem_desc_sw128(kt + (ks >> 2) * (BN * 128) + (ks & 3) * 32,
-                                                              16, 1024),
+                        ptx::umma_f16_ts(tbase + COL_S0 + BN * sb, tbase + COL_Q + 8 * ks,
+                                         dk + (uint64_t)(((ks >> 2) * (BN * 128) + (ks & 3) * 32) >> 4),
                                          id_qk, part > 0 || ks > 0);
                 }
-                ptx::umma_commit(&hd.s_full[b]);
-                if (j >= 1)
-                    ok = issue_pv(j - 1);
+                ptx::umma_commit(&hd.s_full[sb]);
             }
-            if (ok)
-                ok = issue_pv(ntiles - 1);
-            if (!ok)
-                fail();
-            // every committed MMA has finished before TMEM is freed
+            __syncwarp();
+            if (j >= LA)
+                ok = issue_pv(j - LA);
+        }
+        for (int jj = (ntiles > LA ? ntiles - LA : 0); ok && jj < ntiles; ++jj)
+            ok = issue_pv(jj);
+        if (!ok && lane == 0)
+            fail();
+        // every committed MMA has finished before TMEM is freed (a commit tracks all
+        // earlier tcgen05 operations of the issuing thread)
+        if (lane == 0) {
             int none = 0;
-            if (committed >= 0 &&
-                !ptx::mbar_wait_bounded(&hd.pv_done[committed & 1], (committed >> 1) & 1, &none,
-                                        WAIT_NS))
+            if (committed >= 0 && !ptx::mbar_wait_bounded(&hd.pv_done[slot(committed, NS)],
+                                                          par(committed, NS), &none, WAIT_NS))
                 report_timeout(a.status);
         }
+        __syncwarp();
     }
     ptx::tc_fence_before();
     __syncthreads();

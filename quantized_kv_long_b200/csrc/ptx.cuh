@@ -172,6 +172,20 @@ namespace ptx {
 // ---- tcgen05 (5th-generation tensor cores, tensor memory) ---------------------
 // Tensor-memory addresses: bits 31..16 = lane, bits 15..0 = column.
 
+// Warp-collective (all 32 lanes): returns 1 in exactly one lane of the warp.
+// MMAs are issued from warp-converged code by the elected lane: issued from a
+// lone thread inside a lane-divergent branch, a tcgen05.mma costs ~45 cycles
+// to issue whatever its size (measured on B200), so tiles with N < 96 could
+// not keep the tensor pipe busy.
+__device__ __forceinline__ uint32_t elect_one()
+{
+    uint32_t p;
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.u32 %0, 1, 0, e;\n\t}"
+        : "=r"(p));
+    return p;
+}
+
 // Allocate `ncols` TMEM columns (power of two >= 32); the base address is
 // written to shared memory.  Issued by one whole warp.
 __device__ __forceinline__ void tmem_alloc(uint32_t *smem_dst, uint32_t ncols)
