@@ -22,7 +22,7 @@
 //        K^ = d * q as an exact two-part f16 sum (K^hi = RN_f16(d q),
 //        K^lo = fma(d, q, -K^hi)), K-major (keys x head_dim), and
 //        V^ = RN_f16(d * (u - 8)) MN-major (keys x head_dim), zeros past the
-//        end; two slots of each;
+//        end; three slots of each;
 //      - the MMA warp (warp-converged; one elected lane issues) runs
 //        tcgen05.mma: S = Q K^hi^T + Q K^lo^T (A = Q held in tensor memory,
 //        M = 128, N = 32, K = 256, twice) into one of 4 S slots in TMEM --
@@ -66,7 +66,7 @@ constexpr int KROW = 272, VROW = 144;
 constexpr int RAW_K = BN * KROW, RAW_V = BN * VROW, RAW_BYTES = RAW_K + RAW_V;  // 13,312 B
 constexpr int TILE_H = BN * HD * 2;  // one f16 tile of 32 keys x 256 dims: 16 KB
 constexpr int NR = 4;  // raw staging slots (bulk copies in flight ahead of the dequant)
-constexpr int NB = 2;  // f16 K^hi / K^lo / V^ tile slots
+constexpr int NB = 3;  // f16 K^hi / K^lo / V^ tile slots
 constexpr int NS = 4;  // S / P slots in tensor memory
 constexpr int LA = 1;  // the PV of tile j - LA is issued after the QK^T of tile j
 constexpr int N_SOFT = 4, N_DEQ = 8;
