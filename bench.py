@@ -154,10 +154,10 @@ def source_hash(*names: str) -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_record(kernel_files: tuple[str, ...]):
+def traffic_record(kernel_files: tuple[str, ...], record: str = "decode_traffic.json"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the kernel source as it is now (else None)."""
-    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    p = os.path.join(ROOT, "profiles", record)
     try:
         rec = json.load(open(p))
     except Exception:
@@ -317,6 +317,7 @@ def run_ours(args, w: wl.Workload) -> dict | None:
 
 
 DECODE_SOURCES = ("decode.cu", "ptx.cuh", "common.cuh")
+PREFILL_SOURCES = ("prefill.cu", "ptx.cuh", "common.cuh")
 STREAM_METRIC = "q8_0/q4_0 host-streamed decode: H2D GB/s (% of measured H2D), query-tok/s at 262k ctx"
 
 
@@ -488,6 +489,7 @@ def run_prefill(args, w: wl.Workload) -> dict | None:
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
     fl = prefill_flops(w)
     peak, kind = tensor_peak()
+    tr = traffic_record(PREFILL_SOURCES, "prefill_traffic.json")
     cl = clocks.summary()
     res = None
     if rank == 0:
@@ -504,7 +506,8 @@ def run_prefill(args, w: wl.Workload) -> dict | None:
             "roofline": {"bound": "tensor", "kernel": "kvq_prefill_attn (16 layers, 1 launch)",
                          "achieved": round(fl / (k_ms * 1e-3) / 1e12, 2), "peak": peak,
                          "peak_kind": kind, "unit": "TFLOP/s",
-                         "frac": round(fl / (k_ms * 1e-3) / 1e12 / peak, 4), "traffic": None,
+                         "frac": round(fl / (k_ms * 1e-3) / 1e12 / peak, 4),
+                         "traffic": tr["dram_bytes_per_layer"] * L if tr else None,
                          "launch_ms": round(k_ms, 3)},
             "gpu_launches": 2 * args.steps,
             "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
