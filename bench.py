@@ -220,15 +220,26 @@ def run_ours(args, w: wl.Workload) -> dict | None:
 
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+    ws = torch.empty(kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE_STEP, L, Hq, w.n_kv_heads, T, D),
+                     dtype=torch.uint8, device=device)
 
     def step(i=None):
-        kvq.kvq_append(layers, k_new, v_new, n_kv - T, T, stream)
+        if not args.fused:  # append, decode, merge as three launches
+            kvq.kvq_append(layers, k_new, v_new, n_kv - T, T, stream)
+            if i is not None:
+                ev_dec[i][0].record(stream)
+            kvq.kvq_decode_attn(layers, q, Hq, T, n_kv, chunk, w.scale, op, lp, stream)
+            if i is not None:
+                ev_dec[i][1].record(stream)
+            kvq.kvq_merge_lse(op, lp, rows, C, D, out, lse, stream)
+            return
+        # one launch (after clearing its per-head counters): append + decode + merge
         if i is not None:
             ev_dec[i][0].record(stream)
-        kvq.kvq_decode_attn(layers, q, Hq, T, n_kv, chunk, w.scale, op, lp, stream)
+        kvq.kvq_decode_step(layers, k_new, v_new, q, Hq, T, n_kv, chunk, w.scale, op, lp, out,
+                            lse, ws, stream=stream)
         if i is not None:
             ev_dec[i][1].record(stream)
-        kvq.kvq_merge_lse(op, lp, rows, C, D, out, lse, stream)
 
     for _ in range(args.warmup):
         step()
@@ -292,6 +303,8 @@ def run_ours(args, w: wl.Workload) -> dict | None:
         gbs = weak_gbs(world, kv_bytes, ms)
         achieved = kv_bytes / (dec_ms_max * 1e-3) / 1e9
         tr = traffic_record(DECODE_SOURCES)
+        if tr is not None and bool(tr.get("fused", False)) != args.fused:
+            tr = None  # the record is of the other launch sequence
         res = {
             "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
@@ -301,18 +314,23 @@ def run_ours(args, w: wl.Workload) -> dict | None:
                        "head_dim": D, "context": n_kv, "query_tokens": T, "chunk": chunk,
                        "seed": w.seed, "kv_bytes_per_step": kv_bytes,
                        "l2": "inputs larger than L2 (7 GB cache vs 126 MB)",
+                       "step": ("append, decode, merge: 3 launches" if not args.fused else
+                                "kvq_decode_step: 1 launch (+ a 256-byte memset)"),
                        "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
             "query_tok_per_s": round(world * L * T / (ms * 1e-3), 1),
             "pct_hbm_peak": round(100 * gbs / world / peak, 2),
             "e2e": {"value": round(weak_gbs(world, kv_bytes, e2e_ms), 1), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 4)},
-            "roofline": {"bound": "hbm", "kernel": "kvq_decode_attn (16 layers, 1 launch)",
+            "roofline": {"bound": "hbm",
+                         "kernel": ("kvq_decode_attn (16 layers, 1 launch)" if not args.fused else
+                                    "kvq_decode_step: append + decode + merge of 16 layers, "
+                                    "1 launch"),
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": tr["dram_bytes_per_launch"] if tr else None,
                          "launch_ms": round(dec_ms_max, 4)},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (1 if args.fused else 3) * args.steps,
             "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
                        "reasons": cl["reasons"], "samples": cl["samples"]},
         }
@@ -322,7 +340,7 @@ def run_ours(args, w: wl.Workload) -> dict | None:
     return res
 
 
-DECODE_SOURCES = ("decode.cu", "ptx.cuh", "common.cuh")
+DECODE_SOURCES = ("decode.cu", "ptx.cuh", "common.cuh", "merge.cuh", "quant.cuh")
 PREFILL_SOURCES = ("prefill.cu", "ptx.cuh", "common.cuh")
 STREAM_METRIC = "q8_0/q4_0 host-streamed decode: H2D GB/s (% of measured H2D), query-tok/s at 262k ctx"
 
@@ -607,6 +625,9 @@ def main(argv=None) -> int:
     ap.add_argument("--config", default="verify262k",
                     choices=["verify262k", "decode65k", "tiny", "prefill262k", "stream262k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="decode configs: time the step as one kvq_decode_step launch "
+                         "(default: append, decode and merge as three launches)")
     ap.add_argument("--layers", type=int, default=None,
                     help="profile a smaller case of the same kernel: only this many layers")
     args = ap.parse_args(argv)

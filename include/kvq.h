@@ -187,6 +187,41 @@ kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t r
                          kvq_stream stream);
 
 /* ---------------------------------------------------------------------- */
+/* Fused decode step                                                       */
+/* ---------------------------------------------------------------------- */
+
+/* One decode step of all layers in one kernel launch:
+ *   kvq_append(layers, k_new, v_new, pos = n_kv - T, T), then
+ *   kvq_decode_attn(...), then kvq_merge_lse(...)
+ * with the same results (cache bytes, out_part, lse_part, out, lse) as those
+ * three calls.  Inside the launch, the CTA whose chunk holds a new row
+ * quantizes it before reading the chunk, and the last CTA of each
+ * (layer, KV head) to finish merges that head's chunk partials while they
+ * are still in L2; the merge kernel's launch and its re-read of the partials
+ * from memory go away.  Source: the ROCm adaptive KV-streaming page, the
+ * paragraph on the fork's RDNA kernel work (single-queue async graphs,
+ * persistent graph arenas): a decode step as one queue submission.
+ *  k_new, v_new  device fp32 [n_layers][T][n_kv_heads][head_dim], 16-B aligned
+ *  n_kv          keys after the append (the new rows are [n_kv - T, n_kv))
+ *  q, out_part, lse_part, out, lse, chunk, scale: as kvq_decode_attn and
+ *                kvq_merge_lse (rows = n_layers * T * n_q_heads)
+ *  workspace     device, 4-B aligned, >= kvq_workspace_bytes(KVQ_OP_DECODE_STEP,
+ *                ...) = n_layers * n_kv_heads * 4 bytes: per-head counters,
+ *                cleared by the call itself (a cudaMemsetAsync on `stream`
+ *                before the kernel); owned by the caller, not used after the
+ *                step completes
+ * Shapes outside the tiled decode kernel (head_dim != 256, or more than 24
+ * rows per KV head) run the same step as three launches (append, decode,
+ * merge).
+ * Errors: those of kvq_append, kvq_decode_attn and kvq_merge_lse; WORKSPACE
+ *         (null, too small or misaligned workspace). */
+kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k_new,
+                           const float *v_new, const uint16_t *q, int n_q_heads, int T,
+                           int64_t n_kv, int chunk, float scale, float *out_part,
+                           float *lse_part, float *out, float *lse, void *workspace,
+                           size_t ws_bytes, kvq_stream stream);
+
+/* ---------------------------------------------------------------------- */
 /* Chunked prefill                                                         */
 /* ---------------------------------------------------------------------- */
 
@@ -292,9 +327,11 @@ kvq_status kvq_decode_merged_static(const kvq_layer *layers, int n_layers, const
 
 #define KVQ_OP_DECODE 1
 #define KVQ_OP_PREFILL 2
+#define KVQ_OP_DECODE_STEP 3
 
 /* Bytes of device workspace an operation needs (0 if none).
  * KVQ_OP_DECODE: always 0.  KVQ_OP_PREFILL: n_layers, n_q_heads, T as the call.
+ * KVQ_OP_DECODE_STEP: n_layers * n_kv_heads * 4.
  * Returns (size_t)-1 for an unknown op. */
 size_t kvq_workspace_bytes(int op, int n_layers, int n_q_heads, int n_kv_heads, int T,
                            int head_dim);

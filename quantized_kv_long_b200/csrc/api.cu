@@ -151,11 +151,11 @@ kvq_status validate_decode(const kvq_layer *layers, int n_layers, const uint16_t
     return KVQ_OK;
 }
 
-kvq_status enqueue_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
-                          int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
-                          float *out_part, float *lse_part, cudaStream_t s)
+static kvq_status fill_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                              int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                              float *out_part, float *lse_part, DecodeArgs &a)
 {
-    DecodeArgs a;
+    a = DecodeArgs{};
     fill_table(layers, n_layers, a.layers);
     a.n_layers = n_layers;
     a.n_kv_heads = layers[0].n_kv_heads;
@@ -174,6 +174,17 @@ kvq_status enqueue_decode(const kvq_layer *layers, int n_layers, const uint16_t 
     a.force_simple = ks && strcmp(ks, "simple") == 0;
     const char *tt = getenv("KVQ_TEST_DECODE_TIMEOUT");
     a.test_timeout = tt && atoi(tt) != 0;
+    return KVQ_OK;
+}
+
+// Shared by kvq_decode_attn, kvq_stream_decode and kvq_decode_merged_static.
+kvq_status enqueue_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                          int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                          float *out_part, float *lse_part, cudaStream_t s)
+{
+    DecodeArgs a;
+    KVQ_TRY(fill_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
+                        lse_part, a));
     if (!launch_decode(a, s))
         return set_error(KVQ_ERR_UNSUPPORTED, "kvq_decode_attn: no kernel for this shape");
     return check_launch("kvq_decode_attn");
@@ -280,6 +291,54 @@ kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t r
     return check_launch(fn);
 }
 
+kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k_new,
+                           const float *v_new, const uint16_t *q, int n_q_heads, int T,
+                           int64_t n_kv, int chunk, float scale, float *out_part,
+                           float *lse_part, float *out, float *lse, void *workspace,
+                           size_t ws_bytes, kvq_stream stream)
+{
+    const char *fn = "kvq_decode_step";
+    KVQ_TRY(validate_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
+                            lse_part, fn));
+    KVQ_TRY(need(k_new, 16, "k_new", fn));
+    KVQ_TRY(need(v_new, 16, "v_new", fn));
+    const int H = layers[0].n_kv_heads, D = layers[0].head_dim;
+    const int64_t rows = (int64_t)n_layers * T * n_q_heads;
+    const int n_chunks = (int)((n_kv + chunk - 1) / chunk);
+    KVQ_TRY(validate_merge(out_part, lse_part, rows, n_chunks, D, out, lse, fn));
+    const size_t ws_need = kvq_workspace_bytes(KVQ_OP_DECODE_STEP, n_layers, n_q_heads, H, T, D);
+    if (!workspace || ws_bytes < ws_need || !aligned(workspace, 4))
+        return set_error(KVQ_ERR_WORKSPACE,
+                         "%s: needs a 4-byte aligned workspace of %zu bytes (got %zu at %p)", fn,
+                         ws_need, ws_bytes, workspace);
+    const cudaStream_t s = as_stream(stream);
+    DecodeArgs a;
+    KVQ_TRY(fill_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
+                        lse_part, a));
+    if (!a.force_simple && decode_tc_supported(a)) {
+        // one launch: append, decode, and the merge in the last CTA of each (layer, KV head)
+        const cudaError_t e = cudaMemsetAsync(workspace, 0, ws_need, s);
+        if (e != cudaSuccess)
+            return set_error(KVQ_ERR_CUDA, "%s: clearing the workspace: %s", fn,
+                             cudaGetErrorString(e));
+        a.k_new = k_new;
+        a.v_new = v_new;
+        a.out = out;
+        a.lse = lse;
+        a.counters = static_cast<unsigned int *>(workspace);
+        if (!launch_decode(a, s))
+            return set_error(KVQ_ERR_UNSUPPORTED, "%s: no fused kernel for this shape", fn);
+        return check_launch(fn);
+    }
+    // other shapes: the same step as three launches
+    KVQ_TRY(kvq_append(layers, n_layers, k_new, v_new, n_kv - T, T, stream));
+    if (!launch_decode(a, s))
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: no kernel for this shape", fn);
+    KVQ_TRY(check_launch(fn));
+    launch_merge_lse(out_part, lse_part, rows, n_chunks, D, out, lse, s);
+    return check_launch(fn);
+}
+
 kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
                             int n_q_heads, int T, int64_t n_cached, int page, float scale,
                             float *out, float *lse, float *page_out, float *page_lse,
@@ -351,6 +410,10 @@ size_t kvq_workspace_bytes(int op, int n_layers, int n_q_heads, int n_kv_heads, 
 {
     if (op == KVQ_OP_DECODE)
         return 0;
+    if (op == KVQ_OP_DECODE_STEP)
+        return (n_layers > 0 && n_kv_heads > 0)
+                   ? (size_t)n_layers * n_kv_heads * sizeof(unsigned int)
+                   : (size_t)-1;
     if (op == KVQ_OP_PREFILL)
         return prefill_workspace_bytes(n_layers, n_q_heads, n_kv_heads, T, head_dim);
     return (size_t)-1;

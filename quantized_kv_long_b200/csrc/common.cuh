@@ -69,9 +69,17 @@ struct DecodeArgs {
     unsigned int *status;  // device status word (bounded waits that ran out)
     int force_simple;      // host test hook: use the general kernel
     int test_timeout;      // host test hook: make the first wait run out
+    // fused step (all null otherwise): append k_new / v_new [layer][T][kv head][head_dim]
+    // at rows [n_kv - T, n_kv) first, and merge the chunk partials of each (layer, kv head)
+    // into out / lse in the last CTA of that head (counters: one zeroed int per head)
+    const float *k_new, *v_new;
+    float *out, *lse;
+    unsigned int *counters;
 };
 // Returns false (and launches nothing) if no kernel supports the shape.
 bool launch_decode(const DecodeArgs &a, cudaStream_t s);
+// The fused step (DecodeArgs::counters set) exists for the shapes of the tiled kernel.
+bool decode_tc_supported(const DecodeArgs &a);
 
 struct PrefillArgs {
     LayerTable layers;

@@ -47,7 +47,9 @@
 // runs out sets the device status word and the CTA falls through without
 // hanging, after waiting (bounded) for its own copies in flight.
 #include "common.cuh"
+#include "merge.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace kvq {
 
@@ -76,9 +78,13 @@ struct __align__(16) DecodeSmem {
     float4 xs[NPAIR][2][2][NT][32];  // partial S exchange [pair][parity][half][n-tile][lane]
     uint2 qf[2][8][NT][32];          // Q^T B-fragments [half][k-step][n-tile][lane]
     float pm[NPAIR][32], pl[NPAIR][32];
+    float red[NPAIR][2];  // fused step: per-group reduction slots of the merge
     uint64_t full[NS], empty[NS], never;
     int abort;
+    int last;             // fused step: this CTA is the last of its (layer, KV head)
 };
+// fused step: chunks whose merge weights fit in the ring, per 64-thread group
+constexpr int FUSED_SMEM_CHUNKS = (int)(NS * STAGE_BYTES / (NPAIR * sizeof(float)));
 
 // Four int8 in a u32 -> two half2 holding the exact integers:
 // (0x64 << 8 | (b ^ 0x80)) is the f16 1152 + b.
@@ -125,7 +131,7 @@ __device__ __forceinline__ uint32_t k_word(const uint8_t *p, bool aligned)
     return ptx::prmt(lds16(p), lds16(p + 2), 0x5410);
 }
 
-template <int NT>
+template <int NT, bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -170,6 +176,29 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs 
             }
             sm.qf[hf2][ks][nt][ln] = v;
         }
+    }
+    if (FUSED) {
+        // append: the new rows [n_kv - T, n_kv) that fall in this chunk are quantized here,
+        // before any copy of the chunk is issued (no other CTA reads them); one warp
+        // per 32-element block, K blocks 0..7 then V blocks 0..7 of each row
+        const int64_t j_lo = max(c0, a.n_kv - a.T), j_hi = c0 + n_tok;
+        const int tasks = j_hi > j_lo ? (int)(j_hi - j_lo) * 16 : 0;
+        uint8_t *kw = const_cast<uint8_t *>(a.layers.k[layer]);
+        uint8_t *vw = const_cast<uint8_t *>(a.layers.v[layer]);
+        for (int task = threadIdx.x >> 5; task < tasks; task += WARPS) {
+            const int64_t j = j_lo + task / 16;
+            const int blk = task % 16, b = blk & 7;
+            const int tok = (int)(j - (a.n_kv - a.T));
+            const int64_t src = (((int64_t)layer * a.T + tok) * a.n_kv_heads + h) * 256 + b * QK +
+                                (threadIdx.x & 31);
+            const int64_t row = (int64_t)h * cap + j;
+            if (blk < 8)
+                warp_quant_q8_0(a.k_new[src], kw + row * KROW + b * Q8_0_BYTES, threadIdx.x & 31);
+            else
+                warp_quant_q4_0(a.v_new[src], vw + row * VROW + b * Q4_0_BYTES, threadIdx.x & 31);
+        }
+        // the blocks just written are read next by bulk copies (the async proxy)
+        asm volatile("fence.proxy.async.global;" ::: "memory");
     }
     __syncthreads();
     volatile int *abort = &sm.abort;
@@ -515,9 +544,37 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs 
         const int64_t row = ((int64_t)layer * a.T + t) * Hq + h * G + gq;
         a.lse_part[row * C + c] = (L > 0.0f) ? (M + log2f(L)) * LN2 : -INFINITY;
     }
+    if (FUSED) {
+        // the last CTA of this (layer, KV head) to finish merges the chunk partials of its
+        // rows, read through L2.  Release: the barrier orders every thread's partial
+        // writes before thread 0's device-scope fence and count; acquire: the last CTA's
+        // thread 0 fences after seeing the count, and the barrier passes that on.
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            const bool last =
+                atomicAdd(&a.counters[layer * a.n_kv_heads + h], 1u) == (unsigned)(C - 1);
+            if (last)
+                __threadfence();
+            sm.last = last;
+        }
+        __syncthreads();
+        if (sm.last) {
+            const int grp = threadIdx.x >> 6, t64 = threadIdx.x & 63;  // group = warp pair
+            float *w_s = C <= FUSED_SMEM_CHUNKS ? reinterpret_cast<float *>(sm.ring) + grp * C
+                                                : nullptr;
+            for (int col = grp; col < R; col += NPAIR) {
+                const int t = col / G, gq = col % G;
+                const int64_t row = ((int64_t)layer * a.T + t) * Hq + h * G + gq;
+                merge_row<true>(a.out_part + row * C * 256, a.lse_part + row * C, C, 256,
+                                a.out + row * 256, a.lse + row, w_s, sm.red[grp], t64,
+                                [grp] { ptx::named_bar_sync(1 + grp, 64); });
+            }
+        }
+    }
 }
 
-template <int NT>
+template <int NT, bool FUSED>
 bool launch_tc(const DecodeArgs &a, cudaStream_t s)
 {
     const size_t smem = sizeof(DecodeSmem<NT>);
@@ -526,7 +583,8 @@ bool launch_tc(const DecodeArgs &a, cudaStream_t s)
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return false;
     if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(decode_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(decode_tc_kernel<NT, FUSED>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return false;
         attr_set[dev] = true;
@@ -535,7 +593,7 @@ bool launch_tc(const DecodeArgs &a, cudaStream_t s)
     const int64_t grid = (int64_t)a.n_layers * a.n_kv_heads * C;
     if (grid >= (1ll << 31))
         return false;
-    decode_tc_kernel<NT><<<(unsigned)grid, THREADS, smem, s>>>(a);
+    decode_tc_kernel<NT, FUSED><<<(unsigned)grid, THREADS, smem, s>>>(a);
     return true;
 }
 
@@ -549,14 +607,24 @@ bool decode_tc_supported(const DecodeArgs &a)
 
 bool launch_decode(const DecodeArgs &a, cudaStream_t s)
 {
+    if (a.counters) {  // fused step: tiled kernel only
+        if (!decode_tc_supported(a))
+            return false;
+        const int nt = ((a.n_q_heads / a.n_kv_heads) * a.T + 7) / 8;
+        if (nt == 1)
+            return launch_tc<1, true>(a, s);
+        if (nt == 2)
+            return launch_tc<2, true>(a, s);
+        return launch_tc<3, true>(a, s);
+    }
     if (!a.force_simple && decode_tc_supported(a)) {
         const int rows = (a.n_q_heads / a.n_kv_heads) * a.T;
         const int nt = (rows + 7) / 8;
         if (nt == 1)
-            return launch_tc<1>(a, s);
+            return launch_tc<1, false>(a, s);
         if (nt == 2)
-            return launch_tc<2>(a, s);
-        return launch_tc<3>(a, s);
+            return launch_tc<2, false>(a, s);
+        return launch_tc<3, false>(a, s);
     }
     return launch_decode_simple(a, s);
 }

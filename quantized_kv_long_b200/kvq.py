@@ -36,6 +36,7 @@ KVQ_ERR_COPY = 6
 KVQ_ERR_WORKSPACE = 7
 KVQ_OP_DECODE = 1
 KVQ_OP_PREFILL = 2
+KVQ_OP_DECODE_STEP = 3
 KVQ_MAX_LAYERS = 64
 KVQ_MAX_DECODE_T = 4
 KVQ_STATIC_SCRATCH_BYTES = 8 << 20
@@ -63,6 +64,8 @@ _SIGS = {
     "kvq_append": ([_LP, _I32, _P, _P, _I64, _I32, _P], _I32),
     "kvq_decode_attn": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P], _I32),
     "kvq_merge_lse": ([_P, _P, _I64, _I32, _I32, _P, _P, _P], _I32),
+    "kvq_decode_step": ([_LP, _I32, _P, _P, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P,
+                         _SZ, _P], _I32),
     "kvq_prefill_attn": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P, _SZ,
                           _P], _I32),
     "kvq_stream_decode": ([_LP, _I32, _LP, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P,
@@ -153,6 +156,18 @@ def kvq_merge_lse(out_part, lse_part, rows: int, n_chunks: int, head_dim: int, o
                   stream=None) -> None:
     _check(_lib.kvq_merge_lse(_ptr(out_part), _ptr(lse_part), rows, n_chunks, head_dim,
                               _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def kvq_decode_step(layers, k_new, v_new, q, n_q_heads: int, T: int, n_kv: int, chunk: int,
+                    scale: float, out_part, lse_part, out, lse, workspace, ws_bytes: int | None = None,
+                    stream=None) -> None:
+    """Append + decode + merge in one launch (see include/kvq.h)."""
+    arr, n = _layers(layers)
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.kvq_decode_step(arr, n, _ptr(k_new), _ptr(v_new), _ptr(q), n_q_heads, T, n_kv,
+                                chunk, scale, _ptr(out_part), _ptr(lse_part), _ptr(out), _ptr(lse),
+                                _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def kvq_prefill_attn(layers, q, n_q_heads: int, T: int, n_cached: int, page: int, scale: float,

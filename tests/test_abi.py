@@ -116,6 +116,35 @@ def test_merge_validation(kvq):
     _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_merge_lse, A, A, 4, 2, 256, A + 4, A, 0)
 
 
+def test_decode_step_validation(kvq):
+    """kvq_decode_step: the decode and merge checks plus k_new / v_new and the workspace
+    (16 layers x 4 KV heads x 4 bytes = 256 bytes here)."""
+    L = [_layer(kvq)] * 16
+    assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE_STEP, 16, 24, 4, 4, 256) == 256
+    ok = dict(k_new=A, v_new=A, q=A, n_q_heads=24, T=4, n_kv=1024, chunk=256, scale=1 / 16,
+              out_part=A, lse_part=A, out=A, lse=A, workspace=A, ws_bytes=256, stream=0)
+
+    def call(**kw):
+        d = dict(ok)
+        d.update(kw)
+        kvq.kvq_decode_step(L, **d)
+
+    def bad(status, **kw):
+        _raises(kvq, status, call, **kw)
+
+    bad(kvq.KVQ_ERR_INVALID_ARG, k_new=None)
+    bad(kvq.KVQ_ERR_ALIGNMENT, v_new=A + 4)
+    bad(kvq.KVQ_ERR_INVALID_ARG, q=None)
+    bad(kvq.KVQ_ERR_UNSUPPORTED, T=5)
+    bad(kvq.KVQ_ERR_INVALID_ARG, n_kv=3)
+    bad(kvq.KVQ_ERR_INVALID_ARG, n_kv=1025)
+    bad(kvq.KVQ_ERR_ALIGNMENT, out=A + 4)
+    bad(kvq.KVQ_ERR_INVALID_ARG, lse=None)
+    bad(kvq.KVQ_ERR_WORKSPACE, workspace=None)
+    bad(kvq.KVQ_ERR_WORKSPACE, ws_bytes=252)
+    bad(kvq.KVQ_ERR_WORKSPACE, workspace=A + 2)
+
+
 def test_prefill_validation(kvq):
     L = _layer(kvq, capacity=4096)
     ok = dict(q=A, n_q_heads=24, T=128, n_cached=1024, page=1024, scale=1 / 16, out=A, lse=A,
