@@ -363,7 +363,9 @@ def h2d_peak(torch, device, nbytes: int) -> float:
 def run_stream(args, w: wl.Workload) -> dict | None:
     """The stream262k step: the 16-layer cache lives in pinned host memory; every
     layer is copied into one of two device slots while the previous layer's
-    decode attention + merge run on the other (kvq_stream_decode)."""
+    decode attention + merge run on the other (kvq_stream_decode).  With
+    --budget-mib, the layers that fit in that much device memory next to the two
+    slots (kvq_resident_layers) stay resident and only the rest are streamed."""
     import torch
     import torch.distributed as dist
     from quantized_kv_long_b200 import kvq
@@ -388,7 +390,19 @@ def run_stream(args, w: wl.Workload) -> dict | None:
         host.k[l].copy_(tmp.k[0])
         host.v[l].copy_(tmp.v[0])
     del tmp
-    slots = kvq.QuantizedKVCache(2, w.n_kv_heads, D, w.capacity, device=device)
+    layer_bytes = w.capacity * KV_BYTES_PER_TOKEN_LAYER(w)  # one layer, all KV heads
+    R = 0
+    if args.budget_mib is not None:
+        R = kvq.kvq_resident_layers(args.budget_mib << 20, L, w.capacity, w.n_kv_heads, D)
+        if R < 0:
+            raise SystemExit(f"--budget-mib {args.budget_mib}: not even the two slots fit")
+    resident = kvq.QuantizedKVCache(R, w.n_kv_heads, D, w.capacity, device=device) if R else None
+    for l in range(R):  # a resident prefix: the plan's layers live on the device
+        resident.k[l].copy_(host.k[l])
+        resident.v[l].copy_(host.v[l])
+    layers = [resident.layer(l) if l < R else host.layer(l) for l in range(L)]
+    slots = (kvq.QuantizedKVCache(2, w.n_kv_heads, D, w.capacity, device=device)
+             if R < L else None)
     q = torch.from_numpy(np.stack([wl.q_rows(w, l) for l in range(L)])).to(device)
     op = torch.empty((T, Hq, C, D), device=device)
     lp = torch.empty((T, Hq, C), device=device)
@@ -396,7 +410,7 @@ def run_stream(args, w: wl.Workload) -> dict | None:
     lse = torch.empty((L, T, Hq), device=device)
 
     def step():
-        kvq.kvq_stream_decode(host, slots, q, Hq, T, n_kv, chunk, w.scale, op, lp, out, lse,
+        kvq.kvq_stream_decode(layers, slots, q, Hq, T, n_kv, chunk, w.scale, op, lp, out, lse,
                               compute=compute, copy=copy)
 
     for _ in range(args.warmup):
@@ -419,8 +433,10 @@ def run_stream(args, w: wl.Workload) -> dict | None:
     peak = h2d_peak(torch, device, kv_bytes // L)
     cl = clocks.summary()
     res = None
+    streamed = (L - R) * kv_bytes // L
     if rank == 0:
         gbs = world * kv_bytes / (ms * 1e-3) / 1e9
+        link = streamed / (ms * 1e-3) / 1e9  # bytes that crossed the link, per GPU
         res = {
             "metric": STREAM_METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
@@ -428,17 +444,21 @@ def run_stream(args, w: wl.Workload) -> dict | None:
             "dtype": "q8_0 K / q4_0 V x f16 q, f32 accumulate", "data": "synthetic",
             "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": w.n_kv_heads,
                        "head_dim": D, "context": n_kv, "query_tokens": T, "chunk": chunk,
-                       "seed": w.seed, "host_cache_bytes": kv_bytes, "slots": 2},
+                       "seed": w.seed, "host_cache_bytes": kv_bytes,
+                       "slots": 2 if R < L else 0, "resident_layers": R,
+                       "device_budget_mib": args.budget_mib,
+                       "device_cache_bytes": (R + (2 if R < L else 0)) * layer_bytes},
             "query_tok_per_s": round(world * L * T / (ms * 1e-3), 2),
             "roofline": {"bound": "h2d", "kernel": "kvq_stream_decode (copy stream)",
-                         "achieved": round(gbs / world, 2), "peak": round(peak, 2),
+                         "achieved": round(link, 2), "peak": round(peak, 2),
                          "peak_kind": "measured pinned H2D, best of 5, one layer's bytes",
-                         "unit": "GB/s", "frac": round(gbs / world / peak, 4), "traffic": None},
+                         "unit": "GB/s", "frac": round(link / peak, 4),
+                         "streamed_bytes_per_step": streamed, "traffic": None},
             "gpu_launches": 2 * L * args.steps,
             "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
                        "reasons": cl["reasons"], "samples": cl["samples"]},
         }
-    del host, slots
+    del host, slots, resident
     if world > 1:
         dist.destroy_process_group()
     return res
@@ -625,6 +645,9 @@ def main(argv=None) -> int:
     ap.add_argument("--config", default="verify262k",
                     choices=["verify262k", "decode65k", "tiny", "prefill262k", "stream262k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--budget-mib", type=int, default=None,
+                    help="stream262k: device memory for the cache; the layers that fit next to "
+                         "the two streaming slots stay resident (default: all streamed)")
     ap.add_argument("--fused", action="store_true",
                     help="decode configs: time the step as one kvq_decode_step launch "
                          "(default: append, decode and merge as three launches)")

@@ -259,21 +259,27 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
 /* Layer-pipelined host streaming                                          */
 /* ---------------------------------------------------------------------- */
 
-/* Decode attention with the cache in pinned host memory.  For each layer L
- * the K and V rows [0, n_kv) of every head are copied with cudaMemcpyAsync on
- * `copy` into device slot L % 2 while layer L-1 computes on `compute` in the
- * other slot; then decode + merge of layer L run on `compute`.  Events order
- * the two streams: the copy into a slot waits until the compute that last
- * read it is done.  Results equal kvq_decode_attn + kvq_merge_lse on a
- * resident cache bit for bit (same kernels, same data).
+/* Decode attention with the cache in pinned host memory, except for layers
+ * kept resident on the device.  Each layer of host_layers is either streamed
+ * (its k and v are PINNED host memory) or resident (both are device memory of
+ * the current device).  The i-th streamed layer's K and V rows [0, n_kv) of
+ * every head are copied with cudaMemcpyAsync on `copy` into device slot i % 2
+ * while the layers before it compute on `compute`; then decode + merge of the
+ * layer run on `compute` from the slot.  A resident layer is decode + merge in
+ * place.  Layers are computed in order.  Events order the two streams: the
+ * copy into a slot waits until the compute that last read it is done.
+ * Results equal kvq_decode_attn + kvq_merge_lse on a resident cache bit for
+ * bit (same kernels, same data).
  * Source: "Online Log-Sum-Exp prefill & pipelined prefetch" of the RX 9070 XT
  * page (layer L+1's transfer overlapped with layer L's compute); "What
  * shipped" of the ROCm streaming page (the whole KV history in host RAM, a
- * bounded GPU working set reused across layers).
- *  host_layers  host array of n_layers kvq_layer whose k/v are PINNED host
- *               memory (cudaHostAlloc / cudaHostRegister)
+ * bounded GPU working set reused across layers, sized to the device memory
+ * left over: the adaptive part; kvq_resident_layers gives how many layers fit).
+ *  host_layers  host array of n_layers kvq_layer: pinned host memory
+ *               (cudaHostAlloc / cudaHostRegister) or device memory, per layer
  *  dev_slots    host array of 2 kvq_layer (device memory), capacity >= n_kv,
- *               same heads/dim as host_layers
+ *               same heads/dim as host_layers; may be NULL if no layer is
+ *               streamed
  *  q            device fp16 bits [n_layers][T][n_q_heads][head_dim]
  *  out_part, lse_part  device scratch for ONE layer's partials:
  *               [T][n_q_heads][n_chunks][head_dim] and [T][n_q_heads][n_chunks]
@@ -287,6 +293,17 @@ kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_layers,
                              int T, int64_t n_kv, int chunk, float scale, float *out_part,
                              float *lse_part, float *out, float *lse, kvq_stream compute,
                              kvq_stream copy);
+
+/* Adaptive residency: how many of n_layers layers (each n_kv_heads x capacity
+ * K and V head-rows at head_dim) can stay resident in budget_bytes of device
+ * memory while the rest stream through kvq_stream_decode's two slots of one
+ * layer each.  n_layers if everything fits (no slots are needed then);
+ * otherwise the largest R <= n_layers - 1 with (R + 2) layers <= budget; -1 if
+ * not even the two slots fit, or for an invalid shape.  Host arithmetic only.
+ * Source: "What shipped" / "Why it matters" of the ROCm streaming page (a
+ * bounded working set streamed from host RAM when the cache does not fit). */
+int kvq_resident_layers(size_t budget_bytes, int n_layers, int64_t capacity, int n_kv_heads,
+                        int head_dim);
 
 /* ---------------------------------------------------------------------- */
 /* Decode + merge without caller-provided scratch                          */

@@ -1,19 +1,24 @@
-// stream.cu -- layer-pipelined host streaming of the KV cache.
+// stream.cu -- layer-pipelined host streaming of the KV cache, with a
+// resident set of layers.
 //
-// The whole cache stays in pinned host memory; two device slots (each one
-// layer's worth of K and V) form a double-buffered working set that is reused
-// across layers.  Layer L's rows are copied into slot L % 2 on the copy stream
-// while the compute stream runs decode attention + LSE merge of layer L-1 on
-// the other slot.  This is the prefetch scheme of the "Online Log-Sum-Exp
-// prefill & pipelined prefetch" item on the RX 9070 XT KV-streaming page
-// (layer L+1's transfer overlaps layer L's compute) with the bounded,
-// reused working set of "What shipped" on the ROCm KV-streaming page.
+// Each layer's cache is either resident (device memory: computed in place)
+// or streamed (pinned host memory).  Two device slots (each one layer's worth
+// of K and V) form a double-buffered working set reused by the streamed
+// layers: the i-th streamed layer's rows are copied into slot i % 2 on the
+// copy stream while the compute stream runs decode attention + LSE merge of
+// the layers before it.  This is the prefetch scheme of the "Online
+// Log-Sum-Exp prefill & pipelined prefetch" item on the RX 9070 XT
+// KV-streaming page (layer L+1's transfer overlaps layer L's compute) with
+// the bounded, reused working set of "What shipped" on the ROCm KV-streaming
+// page; which layers stay resident is the caller's choice for a device-memory
+// budget (kvq_resident_layers gives the count that fits next to the slots).
 //
-// Ordering, per layer L with slot s = L % 2:
-//   copy:    wait freed[s] (compute of layer L-2 is done with slot s)
+// Ordering, per streamed layer L, the i-th streamed one, slot s = i % 2:
+//   copy:    wait freed[s] (compute of streamed layer i-2 is done with slot s)
 //            memcpy2D K rows [0, n_kv) of every head, then V rows
 //            record ready[s]
 //   compute: wait ready[s]; decode; merge into out[L]; record freed[s]
+// A resident layer is decode + merge on the compute stream, in layer order.
 // Before the first copy the copy stream also waits for all work already
 // enqueued on the compute stream, so a previous call's reads of the slots
 // finish before they are overwritten.
@@ -55,14 +60,22 @@ struct Events {
     }
 };
 
-bool is_pinned_host(const void *p)
+// Where a layer's cache lives: 1 = pinned host, 2 = device memory of the current
+// device, 0 = anything else (pageable host memory, another device, unknown).
+int placement(const void *p)
 {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
         cudaGetLastError();
-        return false;
+        return 0;
     }
-    return at.type == cudaMemoryTypeHost;
+    if (at.type == cudaMemoryTypeHost)
+        return 1;
+    int dev = -1;
+    if (at.type == cudaMemoryTypeDevice && cudaGetDevice(&dev) == cudaSuccess &&
+        at.device == dev)
+        return 2;
+    return 0;
 }
 
 int fail_copy_layer()
@@ -88,26 +101,39 @@ extern "C" kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_laye
                                     out_part, lse_part, fn);
     if (st != KVQ_OK)
         return st;
-    if (!dev_slots)
-        return set_error(KVQ_ERR_INVALID_ARG, "%s: dev_slots is NULL", fn);
-    st = validate_decode(dev_slots, 2, q, n_q_heads, T, n_kv, chunk, scale, out_part, lse_part,
-                         fn);
-    if (st != KVQ_OK)
-        return st;
     const int H = host_layers[0].n_kv_heads, D = host_layers[0].head_dim;
-    if (dev_slots[0].n_kv_heads != H || dev_slots[0].head_dim != D)
-        return set_error(KVQ_ERR_INVALID_ARG, "%s: slots and host layers differ in shape", fn);
-    const int G = n_q_heads / H;
     const int64_t rows = (int64_t)T * n_q_heads;
     const int n_chunks = (int)((n_kv + chunk - 1) / chunk);
     st = validate_merge(out_part, lse_part, rows, n_chunks, D, out, lse, fn);
     if (st != KVQ_OK)
         return st;
-    for (int l = 0; l < n_layers; ++l)
-        if (!is_pinned_host(host_layers[l].k) || !is_pinned_host(host_layers[l].v))
-            return set_error(KVQ_ERR_INVALID_ARG, "%s: host layer %d is not pinned host memory",
+    bool resident[KVQ_MAX_LAYERS];
+    int n_streamed = 0;
+    for (int l = 0; l < n_layers; ++l) {
+        const int pk = placement(host_layers[l].k), pv = placement(host_layers[l].v);
+        if (pk == 0 || pv == 0 || pk != pv)
+            return set_error(KVQ_ERR_INVALID_ARG,
+                             "%s: layer %d: K and V must both be pinned host memory or both "
+                             "device memory of the current device",
                              fn, l);
-    (void)G;
+        resident[l] = pk == 2;
+        n_streamed += !resident[l];
+    }
+    if (n_streamed > 0) {
+        if (!dev_slots)
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: dev_slots is NULL", fn);
+        st = validate_decode(dev_slots, 2, q, n_q_heads, T, n_kv, chunk, scale, out_part,
+                             lse_part, fn);
+        if (st != KVQ_OK)
+            return st;
+        if (dev_slots[0].n_kv_heads != H || dev_slots[0].head_dim != D)
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: slots and host layers differ in shape",
+                             fn);
+        for (int s = 0; s < 2; ++s)
+            if (placement(dev_slots[s].k) != 2 || placement(dev_slots[s].v) != 2)
+                return set_error(KVQ_ERR_INVALID_ARG,
+                                 "%s: slot %d is not device memory of the current device", fn, s);
+    }
 
     cudaStream_t cs = as_stream(compute), ps = as_stream(copy);
     Events E;
@@ -119,12 +145,27 @@ extern "C" kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_laye
 
     const int64_t kr = k_row_bytes(D), vr = v_row_bytes(D);
     const int fail_at = fail_copy_layer();
+    int i_streamed = 0;  // streamed layers enqueued so far
     for (int L = 0; L < n_layers; ++L) {
-        const int s = L & 1;
         const kvq_layer &hl = host_layers[L];
+        const uint16_t *ql = q + (size_t)L * rows * D;
+        if (resident[L]) {
+            st = enqueue_decode(&hl, 1, ql, n_q_heads, T, n_kv, chunk, scale, out_part, lse_part,
+                                cs);
+            if (st != KVQ_OK)
+                return st;
+            launch_merge_lse(out_part, lse_part, rows, n_chunks, D, out + (size_t)L * rows * D,
+                             lse + (size_t)L * rows, cs);
+            st = check_launch(fn);
+            if (st != KVQ_OK)
+                return st;
+            continue;
+        }
+        const int s = i_streamed & 1;
         const kvq_layer &sl = dev_slots[s];
-        if (L >= 2 && cudaStreamWaitEvent(ps, freed[s], 0) != cudaSuccess)
+        if (i_streamed >= 2 && cudaStreamWaitEvent(ps, freed[s], 0) != cudaSuccess)
             return set_error(KVQ_ERR_CUDA, "%s: event wait failed", fn);
+        ++i_streamed;
         if (L == fail_at)
             return set_error(KVQ_ERR_COPY, "%s: copy of layer %d failed (test hook)", fn, L);
         cudaError_t e = cudaMemcpy2DAsync(sl.k, (size_t)(sl.capacity * kr), hl.k,
@@ -140,7 +181,6 @@ extern "C" kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_laye
         if (cudaEventRecord(ready[s], ps) != cudaSuccess ||
             cudaStreamWaitEvent(cs, ready[s], 0) != cudaSuccess)
             return set_error(KVQ_ERR_CUDA, "%s: event ordering failed", fn);
-        const uint16_t *ql = q + (size_t)L * rows * D;
         st = enqueue_decode(&sl, 1, ql, n_q_heads, T, n_kv, chunk, scale, out_part, lse_part, cs);
         if (st != KVQ_OK)
             return st;
@@ -153,4 +193,20 @@ extern "C" kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_laye
             return set_error(KVQ_ERR_CUDA, "%s: event record failed", fn);
     }
     return KVQ_OK;
+}
+
+extern "C" int kvq_resident_layers(size_t budget_bytes, int n_layers, int64_t capacity,
+                                   int n_kv_heads, int head_dim)
+{
+    if (n_layers < 1 || capacity < 1 || n_kv_heads < 1 || head_dim < QK || head_dim % QK != 0)
+        return -1;
+    const double layer = (double)n_kv_heads * (double)capacity *
+                         (double)(k_row_bytes(head_dim) + v_row_bytes(head_dim));
+    const double budget = (double)budget_bytes;
+    if (layer * n_layers <= budget)
+        return n_layers;  // everything resident: no slots needed
+    if (2.0 * layer > budget)
+        return -1;  // not even the two streaming slots fit
+    const double r = (budget - 2.0 * layer) / layer;
+    return r >= n_layers - 1 ? n_layers - 1 : (int)r;
 }

@@ -72,6 +72,7 @@ _SIGS = {
                            _P], _I32),
     "kvq_decode_merged_static": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P],
                                  _I32),
+    "kvq_resident_layers": ([_SZ, _I32, _I64, _I32, _I32], _I32),
     "kvq_workspace_bytes": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "kvq_check": ([_P], _I32),
     "kvq_status_string": ([_I32], ctypes.c_char_p),
@@ -183,9 +184,12 @@ def kvq_stream_decode(host_layers, dev_slots, q, n_q_heads: int, T: int, n_kv: i
                       scale: float, out_part, lse_part, out, lse, compute=None,
                       copy=None) -> None:
     harr, n = _layers(host_layers)
-    sarr, ns = _layers(dev_slots)
-    if ns != 2:
-        raise ValueError("dev_slots must hold exactly 2 layers")
+    if dev_slots is None:
+        sarr = None
+    else:
+        sarr, ns = _layers(dev_slots)
+        if ns != 2:
+            raise ValueError("dev_slots must hold exactly 2 layers")
     _check(_lib.kvq_stream_decode(harr, n, sarr, _ptr(q), n_q_heads, T, n_kv, chunk, scale,
                                   _ptr(out_part), _ptr(lse_part), _ptr(out), _ptr(lse),
                                   _stream(compute), _stream(copy)))
@@ -198,6 +202,11 @@ def kvq_decode_merged_static(layers, q, n_q_heads: int, T: int, n_kv: int, chunk
     arr, n = _layers(layers)
     _check(_lib.kvq_decode_merged_static(arr, n, _ptr(q), n_q_heads, T, n_kv, chunk, scale,
                                          _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def kvq_resident_layers(budget_bytes: int, n_layers: int, capacity: int, n_kv_heads: int,
+                        head_dim: int) -> int:
+    return _lib.kvq_resident_layers(budget_bytes, n_layers, capacity, n_kv_heads, head_dim)
 
 
 def kvq_workspace_bytes(op: int, n_layers: int, n_q_heads: int, n_kv_heads: int, T: int,

@@ -174,3 +174,19 @@ def test_stream_validation(kvq):
 def test_workspace_query(kvq):
     assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE, 16, 24, 4, 4, 256) == 0
     assert kvq.kvq_workspace_bytes(99, 1, 1, 1, 1, 32) == ctypes.c_size_t(-1).value
+
+
+def test_resident_layers_plan(kvq):
+    """Host arithmetic of the residency plan: 16 layers x 4 heads x 262,144 tokens
+    x (272 + 144) B = 436,207,616 B per layer."""
+    lb = 4 * 262144 * (272 + 144)
+    plan = lambda budget, n=16: kvq.kvq_resident_layers(budget, n, 262144, 4, 256)
+    assert plan(16 * lb) == 16          # everything fits: no slots
+    assert plan(16 * lb - 1) == 13      # 13 resident + 2 slots = 15 layers of memory
+    assert plan(3 * lb) == 1
+    assert plan(2 * lb) == 0            # only the two slots
+    assert plan(2 * lb - 1) == -1       # not even the slots
+    assert plan(2100 << 20) == 3        # the ~2,100 MiB decode working set of the pages
+    assert plan(10**15, 1) == 1
+    assert kvq.kvq_resident_layers(1 << 40, 0, 1024, 4, 256) == -1
+    assert kvq.kvq_resident_layers(1 << 40, 4, 1024, 4, 48) == -1

@@ -110,3 +110,66 @@ def test_pageable_host_memory_rejected(kvq):
         kvq.kvq_stream_decode(pageable, slots, q, Hq, 1, 64, 64, w.scale, op, lp, out, lse,
                               compute=torch.cuda.current_stream(), copy=torch.cuda.Stream())
     assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
+
+
+def _mixed(kvq, dev, host, pattern):
+    """Layer l from device memory where pattern[l] == 'D', from pinned host memory where 'H'."""
+    return [dev.layer(l) if c == "D" else host.layer(l) for l, c in enumerate(pattern)]
+
+
+@pytest.mark.parametrize("pattern", ["DDHHH", "HDHDH", "DDDDH"])
+def test_resident_layers_mixed_with_streamed(kvq, pattern):
+    """A resident prefix (the plan kvq_resident_layers makes), an interleaving and a
+    single streamed layer: bit-identical to the all-resident path."""
+    n_kv, chunk, T = 5000, 1024, 4
+    w, dev, orc, host, slots, q = _setup(kvq, T=T)
+    Hq, D = w.n_q_heads, w.head_dim
+    C = -(-n_kv // chunk)
+    op = torch.empty((T, Hq, C, D), device="cuda")
+    lp = torch.empty((T, Hq, C), device="cuda")
+    out = torch.full((5, T, Hq, D), float("nan"), device="cuda")
+    lse = torch.full((5, T, Hq), float("nan"), device="cuda")
+    kvq.kvq_stream_decode(_mixed(kvq, dev, host, pattern), slots, q, Hq, T, n_kv, chunk, w.scale,
+                          op, lp, out, lse, compute=torch.cuda.current_stream(),
+                          copy=torch.cuda.Stream())
+    kvq.kvq_check()
+    ro, rl = _resident(kvq, w, dev, q, n_kv, chunk, T)
+    assert np.array_equal(out.cpu().numpy(), ro) and np.array_equal(lse.cpu().numpy(), rl)
+
+
+def test_all_resident_needs_no_slots(kvq):
+    n_kv, chunk = 5000, 1024
+    w, dev, orc, host, slots, q = _setup(kvq, n_layers=3)
+    Hq, D = w.n_q_heads, w.head_dim
+    C = -(-n_kv // chunk)
+    op = torch.empty((1, Hq, C, D), device="cuda")
+    lp = torch.empty((1, Hq, C), device="cuda")
+    out = torch.full((3, 1, Hq, D), float("nan"), device="cuda")
+    lse = torch.full((3, 1, Hq), float("nan"), device="cuda")
+    kvq.kvq_stream_decode(dev.layers(), None, q, Hq, 1, n_kv, chunk, w.scale, op, lp, out, lse,
+                          compute=torch.cuda.current_stream(), copy=torch.cuda.Stream())
+    kvq.kvq_check()
+    ro, rl = _resident(kvq, w, dev, q, n_kv, chunk, 1)
+    assert np.array_equal(out.cpu().numpy(), ro) and np.array_equal(lse.cpu().numpy(), rl)
+    # a streamed layer without slots is refused before anything is enqueued
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_stream_decode(_mixed(kvq, dev, host, "DHD"), None, q, Hq, 1, n_kv, chunk,
+                              w.scale, op, lp, out, lse, compute=torch.cuda.current_stream(),
+                              copy=torch.cuda.Stream())
+    assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_split_placement_rejected(kvq):
+    """K on the device and V in host memory (or the reverse) is not a valid layer."""
+    n_kv, chunk = 64, 64
+    w, dev, orc, host, slots, q = _setup(kvq, n_layers=1, n_kv=n_kv, cap=64)
+    Hq, D = w.n_q_heads, w.head_dim
+    bad = [kvq.kvq_layer(dev.k[0].data_ptr(), host.v[0].data_ptr(), 64, w.n_kv_heads, D)]
+    op = torch.empty((1, Hq, 1, D), device="cuda")
+    lp = torch.empty((1, Hq, 1), device="cuda")
+    out = torch.empty((1, 1, Hq, D), device="cuda")
+    lse = torch.empty((1, 1, Hq), device="cuda")
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_stream_decode(bad, slots, q, Hq, 1, n_kv, chunk, w.scale, op, lp, out, lse,
+                              compute=torch.cuda.current_stream(), copy=torch.cuda.Stream())
+    assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
