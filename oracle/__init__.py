@@ -9,7 +9,11 @@ the header of ``kvq_oracle.c``.
 
 Every function here takes and returns numpy arrays.  Caches use the layout of
 one layer: K ``[n_kv_heads, capacity, head_dim // 32 * 34]`` uint8 and V
-``[n_kv_heads, capacity, head_dim // 32 * 18]`` uint8.
+``[n_kv_heads, capacity, head_dim // 32 * 18]`` uint8 in the main (Q8_0 K /
+Q4_0 V) configuration; either tensor may use the other block format
+(``empty_cache(..., k_fmt=, v_fmt=)``), and the functions read each tensor's
+format from its head-row length (34 or 18 bytes per 32 elements, never both
+for head_dim <= 512).
 
 Parity pins: every function below is pinned by the CPU tests (golden blocks,
 closed forms, library cross-checks, invariants); none is "parity unpinned".
@@ -26,6 +30,8 @@ from .build import build_oracle, library_path
 QK = 32
 Q8_0_BYTES = 34
 Q4_0_BYTES = 18
+FMT_Q8_0, FMT_Q4_0 = 1, 2
+_BLOCK_BYTES = {FMT_Q8_0: Q8_0_BYTES, FMT_Q4_0: Q4_0_BYTES}
 
 _lib = None
 
@@ -49,12 +55,14 @@ def _load():
         "orc_quantize_q4_0": ([P, P, i64], None),
         "orc_dequant_q8_0": ([P, P, i64], None),
         "orc_dequant_q4_0": ([P, P, i64], None),
-        "orc_append": ([P, P, i32, i32, i64, P, P, i64, i64], None),
-        "orc_decode_attn": ([P, P, i32, i32, i64, P, i32, i32, i64, i64, f64, P, P], None),
+        "orc_append": ([P, P, i32, i32, i64, P, P, i64, i64, i32, i32], None),
+        "orc_decode_attn": ([P, P, i32, i32, i64, P, i32, i32, i64, i64, f64, P, P, i32, i32],
+                            None),
         "orc_merge_lse": ([P, P, i64, i32, i32, P, P], None),
-        "orc_attn_rows": ([P, P, i32, i32, i64, P, P, i32, P, P, i64, f64, P, P], None),
-        "orc_prefill_attn": ([P, P, i32, i32, i64, P, i32, i32, i64, i64, f64, P, P, P, P],
-                             None),
+        "orc_attn_rows": ([P, P, i32, i32, i64, P, P, i32, P, P, i64, f64, P, P, i32, i32],
+                          None),
+        "orc_prefill_attn": ([P, P, i32, i32, i64, P, i32, i32, i64, i64, f64, P, P, P, P, i32,
+                              i32], None),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -132,32 +140,44 @@ def dequant_q4_0(b: np.ndarray) -> np.ndarray:
 
 # ---- cache ------------------------------------------------------------------
 
-def empty_cache(n_kv_heads: int, head_dim: int, capacity: int):
-    """Zeroed K and V byte arrays of one layer."""
-    k = np.zeros((n_kv_heads, capacity, head_dim // QK * Q8_0_BYTES), dtype=np.uint8)
-    v = np.zeros((n_kv_heads, capacity, head_dim // QK * Q4_0_BYTES), dtype=np.uint8)
+def empty_cache(n_kv_heads: int, head_dim: int, capacity: int, k_fmt: int = FMT_Q8_0,
+                v_fmt: int = FMT_Q4_0):
+    """Zeroed K and V byte arrays of one layer (K blocks in ``k_fmt``, V in ``v_fmt``)."""
+    k = np.zeros((n_kv_heads, capacity, head_dim // QK * _BLOCK_BYTES[k_fmt]), dtype=np.uint8)
+    v = np.zeros((n_kv_heads, capacity, head_dim // QK * _BLOCK_BYTES[v_fmt]), dtype=np.uint8)
     return k, v
+
+
+def _fmt_dim(row_bytes: int) -> tuple[int, int]:
+    """(block format, head_dim) of a head-row of ``row_bytes``: exactly one of the two
+    formats fits when head_dim <= 512."""
+    fits = [(f, row_bytes // b * QK) for f, b in _BLOCK_BYTES.items()
+            if row_bytes % b == 0 and row_bytes // b * QK <= 512]
+    assert len(fits) == 1, f"head-row of {row_bytes} bytes"
+    return fits[0]
+
+
+def _cache_dims(k_cache, v_cache):
+    """(n_kv_heads, head_dim, capacity, k_fmt, v_fmt) of one layer's caches."""
+    H, cap, kb = k_cache.shape
+    k_fmt, D = _fmt_dim(kb)
+    v_fmt, Dv = _fmt_dim(v_cache.shape[2])
+    assert v_cache.shape[:2] == (H, cap) and Dv == D
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    return H, D, cap, k_fmt, v_fmt
 
 
 def append(k_cache, v_cache, k_new, v_new, pos: int) -> None:
     """Quantize rows ``k_new``/``v_new`` ``[n_tok, n_kv_heads, head_dim]`` into rows
     ``[pos, pos + n_tok)`` of the caches, in place."""
-    H, cap, _ = k_cache.shape
+    H, D0, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache)
     k_new = np.ascontiguousarray(k_new, dtype=np.float32)
     v_new = np.ascontiguousarray(v_new, dtype=np.float32)
     n_tok, h2, D = k_new.shape
-    if h2 != H or v_new.shape != k_new.shape or pos < 0 or pos + n_tok > cap:
+    if h2 != H or D != D0 or v_new.shape != k_new.shape or pos < 0 or pos + n_tok > cap:
         raise ValueError("bad append shape")
     _load().orc_append(_ptr(k_cache), _ptr(v_cache), H, D, cap, _ptr(k_new), _ptr(v_new),
-                       pos, n_tok)
-
-
-def _cache_dims(k_cache, v_cache):
-    H, cap, kb = k_cache.shape
-    D = kb // Q8_0_BYTES * QK
-    assert v_cache.shape == (H, cap, D // QK * Q4_0_BYTES)
-    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
-    return H, D, cap
+                       pos, n_tok, k_fmt, v_fmt)
 
 
 # ---- attention --------------------------------------------------------------
@@ -167,7 +187,7 @@ def decode_attn(k_cache, v_cache, q: np.ndarray, n_kv: int, chunk: int, scale: f
 
     Returns ``(out_part [T, Hq, n_chunks, D] f64, lse_part [T, Hq, n_chunks] f64)``.
     """
-    H, D, cap = _cache_dims(k_cache, v_cache)
+    H, D, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache)
     q = np.ascontiguousarray(q, dtype=np.float16)
     T, Hq, D2 = q.shape
     assert D2 == D and Hq % H == 0 and 1 <= T <= n_kv <= cap and chunk >= 1
@@ -175,7 +195,7 @@ def decode_attn(k_cache, v_cache, q: np.ndarray, n_kv: int, chunk: int, scale: f
     out = np.empty((T, Hq, n_chunks, D), dtype=np.float64)
     lse = np.empty((T, Hq, n_chunks), dtype=np.float64)
     _load().orc_decode_attn(_ptr(k_cache), _ptr(v_cache), H, D, cap, _ptr(q.view(np.uint16)),
-                            Hq, T, n_kv, chunk, scale, _ptr(out), _ptr(lse))
+                            Hq, T, n_kv, chunk, scale, _ptr(out), _ptr(lse), k_fmt, v_fmt)
     return out, lse
 
 
@@ -195,7 +215,7 @@ def merge_lse(out_part: np.ndarray, lse_part: np.ndarray):
 def attn_rows(k_cache, v_cache, q_rows: np.ndarray, q_head: np.ndarray, n_q_heads: int,
               key_begin: np.ndarray, key_end: np.ndarray, scale: float):
     """One-pass attention of arbitrary rows (fp16 ``q_rows [n, D]``)."""
-    H, D, cap = _cache_dims(k_cache, v_cache)
+    H, D, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache)
     q_rows = np.ascontiguousarray(q_rows, dtype=np.float16)
     n = q_rows.shape[0]
     q_head = np.ascontiguousarray(q_head, dtype=np.int32)
@@ -207,7 +227,7 @@ def attn_rows(k_cache, v_cache, q_rows: np.ndarray, q_head: np.ndarray, n_q_head
     lse = np.empty(n, dtype=np.float64)
     _load().orc_attn_rows(_ptr(k_cache), _ptr(v_cache), H, D, cap,
                           _ptr(q_rows.view(np.uint16)), _ptr(q_head), n_q_heads, _ptr(kb),
-                          _ptr(ke), n, scale, _ptr(out), _ptr(lse))
+                          _ptr(ke), n, scale, _ptr(out), _ptr(lse), k_fmt, v_fmt)
     return out, lse
 
 
@@ -218,7 +238,7 @@ def prefill_attn(k_cache, v_cache, q: np.ndarray, n_cached: int, page: int, scal
     Returns ``(out [T, Hq, D], lse [T, Hq])`` and, with ``pages=True``, also
     ``(page_out [T, Hq, n_pages, D], page_lse [T, Hq, n_pages])``.
     """
-    H, D, cap = _cache_dims(k_cache, v_cache)
+    H, D, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache)
     q = np.ascontiguousarray(q, dtype=np.float16)
     T, Hq, _ = q.shape
     assert n_cached + T <= cap and Hq % H == 0
@@ -229,5 +249,5 @@ def prefill_attn(k_cache, v_cache, q: np.ndarray, n_cached: int, page: int, scal
     pl = np.empty((T, Hq, n_pages), dtype=np.float64) if pages else None
     _load().orc_prefill_attn(_ptr(k_cache), _ptr(v_cache), H, D, cap,
                              _ptr(q.view(np.uint16)), Hq, T, n_cached, page, scale, _ptr(out),
-                             _ptr(lse), _ptr(po), _ptr(pl))
+                             _ptr(lse), _ptr(po), _ptr(pl), k_fmt, v_fmt)
     return (out, lse, po, pl) if pages else (out, lse)

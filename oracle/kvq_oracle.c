@@ -49,6 +49,10 @@
  * Cache layout of one layer (the interface both sides implement):
  *   K: [n_kv_heads][capacity][head_dim/32] Q8_0 blocks (34 B each)
  *   V: [n_kv_heads][capacity][head_dim/32] Q4_0 blocks (18 B each)
+ * The pages' main configuration.  Each tensor may also use the other format
+ * (q8_0/q8_0 and q4_0/q4_0 caches are the other choices of the KV-cache
+ * guide's levers section): the cache functions take the block format of K and
+ * of V (FMT_Q8_0 or FMT_Q4_0), and a head-row is head_dim/32 blocks of it.
  *
  * Build: gcc -std=c11 -O2 -fopenmp -ffp-contract=off -fPIC -shared.
  * Floating-point contraction must stay off: the quantizers are defined as a
@@ -65,6 +69,8 @@
 #define QK 32
 #define Q8_0_BYTES 34
 #define Q4_0_BYTES 18
+#define FMT_Q8_0 1
+#define FMT_Q4_0 2
 
 /* ------------------------------------------------------------------------ */
 /* fp16 <-> fp32, written from the IEEE 754 binary16 definition.            */
@@ -238,40 +244,56 @@ void orc_dequant_q4_0(const uint8_t *blocks, double *x, int64_t n)
 }
 
 /* ------------------------------------------------------------------------ */
-/* Cache layout helpers                                                     */
+/* Cache layout helpers: a block format is FMT_Q8_0 or FMT_Q4_0             */
 /* ------------------------------------------------------------------------ */
 
-static size_t k_row_bytes(int head_dim) { return (size_t)(head_dim / QK) * Q8_0_BYTES; }
-static size_t v_row_bytes(int head_dim) { return (size_t)(head_dim / QK) * Q4_0_BYTES; }
+static size_t block_bytes(int fmt) { return fmt == FMT_Q8_0 ? Q8_0_BYTES : Q4_0_BYTES; }
 
-static const uint8_t *k_row(const uint8_t *k_cache, int head_dim, int64_t capacity, int h,
-                            int64_t j)
+static size_t row_bytes(int fmt, int head_dim) { return (size_t)(head_dim / QK) * block_bytes(fmt); }
+
+static void quant_block(int fmt, const float *x, uint8_t *b)
 {
-    return k_cache + ((size_t)h * (size_t)capacity + (size_t)j) * k_row_bytes(head_dim);
+    if (fmt == FMT_Q8_0)
+        quant_block_q8_0(x, b);
+    else
+        quant_block_q4_0(x, b);
 }
 
-static const uint8_t *v_row(const uint8_t *v_cache, int head_dim, int64_t capacity, int h,
-                            int64_t j)
+static void dequant_block(int fmt, const uint8_t *b, double *y)
 {
-    return v_cache + ((size_t)h * (size_t)capacity + (size_t)j) * v_row_bytes(head_dim);
+    if (fmt == FMT_Q8_0)
+        dequant_block_q8_0(b, y);
+    else
+        dequant_block_q4_0(b, y);
+}
+
+/* Head-row j of KV head h, dequantized into y[0..head_dim). */
+static void dequant_row(const uint8_t *cache, int fmt, int head_dim, int64_t capacity, int h,
+                        int64_t j, double *y)
+{
+    const uint8_t *r = cache + ((size_t)h * (size_t)capacity + (size_t)j) * row_bytes(fmt, head_dim);
+    for (int b = 0; b < head_dim / QK; ++b)
+        dequant_block(fmt, r + b * block_bytes(fmt), y + b * QK);
 }
 
 /* Quantize-on-append: rows [pos, pos+n_tok) of every KV head.  k_new and
- * v_new are fp32 [n_tok][n_kv_heads][head_dim]. */
+ * v_new are fp32 [n_tok][n_kv_heads][head_dim]; K blocks in format k_fmt, V
+ * blocks in format v_fmt. */
 void orc_append(uint8_t *k_cache, uint8_t *v_cache, int n_kv_heads, int head_dim,
                 int64_t capacity, const float *k_new, const float *v_new, int64_t pos,
-                int64_t n_tok)
+                int64_t n_tok, int k_fmt, int v_fmt)
 {
 #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t t = 0; t < n_tok; ++t)
         for (int h = 0; h < n_kv_heads; ++h) {
             const float *ks = k_new + ((size_t)t * n_kv_heads + h) * head_dim;
             const float *vs = v_new + ((size_t)t * n_kv_heads + h) * head_dim;
-            uint8_t *kd = k_cache + ((size_t)h * capacity + (size_t)(pos + t)) * k_row_bytes(head_dim);
-            uint8_t *vd = v_cache + ((size_t)h * capacity + (size_t)(pos + t)) * v_row_bytes(head_dim);
+            const size_t row = (size_t)h * capacity + (size_t)(pos + t);
+            uint8_t *kd = k_cache + row * row_bytes(k_fmt, head_dim);
+            uint8_t *vd = v_cache + row * row_bytes(v_fmt, head_dim);
             for (int b = 0; b < head_dim / QK; ++b) {
-                quant_block_q8_0(ks + b * QK, kd + b * Q8_0_BYTES);
-                quant_block_q4_0(vs + b * QK, vd + b * Q4_0_BYTES);
+                quant_block(k_fmt, ks + b * QK, kd + b * block_bytes(k_fmt));
+                quant_block(v_fmt, vs + b * QK, vd + b * block_bytes(v_fmt));
             }
         }
 }
@@ -285,9 +307,9 @@ void orc_append(uint8_t *k_cache, uint8_t *v_cache, int n_kv_heads, int head_dim
  * for every visible key are computed first; the max is taken over those
  * complete scores, then the weights, their sum, the output and the lse.
  * Results: out [n_rows][head_dim], lse [n_rows]. */
-static void attend(const uint8_t *k_cache, const uint8_t *v_cache, int head_dim,
-                   int64_t capacity, int h, const double *q, int n_rows, const int64_t *k0,
-                   const int64_t *k1, double scale, double *out, double *lse)
+static void attend(const uint8_t *k_cache, const uint8_t *v_cache, int k_fmt, int v_fmt,
+                   int head_dim, int64_t capacity, int h, const double *q, int n_rows,
+                   const int64_t *k0, const int64_t *k1, double scale, double *out, double *lse)
 {
     int64_t lo = INT64_MAX, hi = INT64_MIN;
     for (int r = 0; r < n_rows; ++r) {
@@ -311,9 +333,7 @@ static void attend(const uint8_t *k_cache, const uint8_t *v_cache, int head_dim,
 
     /* 1. complete scores */
     for (int64_t j = lo; j < hi; ++j) {
-        const uint8_t *kr = k_row(k_cache, head_dim, capacity, h, j);
-        for (int b = 0; b < head_dim / QK; ++b)
-            dequant_block_q8_0(kr + b * Q8_0_BYTES, kh + b * QK);
+        dequant_row(k_cache, k_fmt, head_dim, capacity, h, j, kh);
         for (int r = 0; r < n_rows; ++r) {
             double acc = 0.0;
             const double *qr = q + (size_t)r * head_dim;
@@ -334,9 +354,7 @@ static void attend(const uint8_t *k_cache, const uint8_t *v_cache, int head_dim,
     }
     /* 3. weights, their sum and the weighted V sum */
     for (int64_t j = lo; j < hi; ++j) {
-        const uint8_t *vr = v_row(v_cache, head_dim, capacity, h, j);
-        for (int b = 0; b < head_dim / QK; ++b)
-            dequant_block_q4_0(vr + b * Q4_0_BYTES, vh + b * QK);
+        dequant_row(v_cache, v_fmt, head_dim, capacity, h, j, vh);
         for (int r = 0; r < n_rows; ++r) {
             if (j < k0[r] || j >= k1[r])
                 continue;
@@ -378,7 +396,7 @@ static void load_q(const uint16_t *q16, double *q, int64_t n)
 void orc_decode_attn(const uint8_t *k_cache, const uint8_t *v_cache, int n_kv_heads,
                      int head_dim, int64_t capacity, const uint16_t *q, int n_q_heads, int T,
                      int64_t n_kv, int64_t chunk, double scale, double *out_part,
-                     double *lse_part)
+                     double *lse_part, int k_fmt, int v_fmt)
 {
     int G = n_q_heads / n_kv_heads;
     int64_t n_chunks = (n_kv + chunk - 1) / chunk;
@@ -401,7 +419,8 @@ void orc_decode_attn(const uint8_t *k_cache, const uint8_t *v_cache, int n_kv_he
                     k0[r] = c0;
                     k1[r] = (last + 1 < c1) ? last + 1 : c1;
                 }
-            attend(k_cache, v_cache, head_dim, capacity, h, qd, rows, k0, k1, scale, o, ls);
+            attend(k_cache, v_cache, k_fmt, v_fmt, head_dim, capacity, h, qd, rows, k0, k1,
+                   scale, o, ls);
             for (int t = 0; t < T; ++t)
                 for (int g = 0; g < G; ++g) {
                     int r = t * G + g, qh = h * G + g;
@@ -460,15 +479,15 @@ void orc_attn_rows(const uint8_t *k_cache, const uint8_t *v_cache, int n_kv_head
                    int head_dim, int64_t capacity, const uint16_t *q_rows,
                    const int32_t *q_head, int n_q_heads, const int64_t *key_begin,
                    const int64_t *key_end, int64_t n_rows, double scale, double *out,
-                   double *lse)
+                   double *lse, int k_fmt, int v_fmt)
 {
     int G = n_q_heads / n_kv_heads;
 #pragma omp parallel for schedule(dynamic)
     for (int64_t r = 0; r < n_rows; ++r) {
         double *qd = (double *)malloc(sizeof(double) * head_dim);
         load_q(q_rows + (size_t)r * head_dim, qd, head_dim);
-        attend(k_cache, v_cache, head_dim, capacity, q_head[r] / G, qd, 1, key_begin + r,
-               key_end + r, scale, out + (size_t)r * head_dim, lse + r);
+        attend(k_cache, v_cache, k_fmt, v_fmt, head_dim, capacity, q_head[r] / G, qd, 1,
+               key_begin + r, key_end + r, scale, out + (size_t)r * head_dim, lse + r);
         free(qd);
     }
 }
@@ -482,7 +501,7 @@ void orc_attn_rows(const uint8_t *k_cache, const uint8_t *v_cache, int n_kv_head
 void orc_prefill_attn(const uint8_t *k_cache, const uint8_t *v_cache, int n_kv_heads,
                       int head_dim, int64_t capacity, const uint16_t *q, int n_q_heads, int T,
                       int64_t n_cached, int64_t page, double scale, double *out, double *lse,
-                      double *page_out, double *page_lse)
+                      double *page_out, double *page_lse, int k_fmt, int v_fmt)
 {
     int G = n_q_heads / n_kv_heads;
     int64_t n_keys = n_cached + T;
@@ -494,15 +513,15 @@ void orc_prefill_attn(const uint8_t *k_cache, const uint8_t *v_cache, int n_kv_h
             load_q(q + ((size_t)t * n_q_heads + qh) * head_dim, qd, head_dim);
             size_t row = (size_t)t * n_q_heads + qh;
             int64_t b = 0, e = n_cached + t + 1;
-            attend(k_cache, v_cache, head_dim, capacity, qh / G, qd, 1, &b, &e, scale,
-                   out + row * head_dim, lse + row);
+            attend(k_cache, v_cache, k_fmt, v_fmt, head_dim, capacity, qh / G, qd, 1, &b, &e,
+                   scale, out + row * head_dim, lse + row);
             if (page_out) {
                 for (int64_t p = 0; p < n_pages; ++p) {
                     int64_t p0 = p * page, p1 = p0 + page < e ? p0 + page : e;
                     if (p1 < p0)
                         p1 = p0;
-                    attend(k_cache, v_cache, head_dim, capacity, qh / G, qd, 1, &p0, &p1,
-                           scale, page_out + (row * n_pages + p) * head_dim,
+                    attend(k_cache, v_cache, k_fmt, v_fmt, head_dim, capacity, qh / G, qd, 1,
+                           &p0, &p1, scale, page_out + (row * n_pages + p) * head_dim,
                            page_lse + row * n_pages + p);
                 }
             }

@@ -219,3 +219,61 @@ def test_workload_generator_is_seeded_and_blockwise():
     q = wl.q_rows(w, 0)
     assert q.dtype == np.float16 and q.shape == (1, 24, 256)
     assert not np.array_equal(wl.kv_rows(w, 0, 1, 0, 10), a[:10])
+
+
+# ------------------------------------------------------- other block formats
+# The KV-cache guide's levers section lists q8_0 and q4_0 caches for both
+# tensors.  The format plumbing (which block format each tensor's rows are
+# written and read in) is pinned against the separately pinned block
+# quantizers and dequantizers.
+
+FORMATS = [(oracle.FMT_Q8_0, oracle.FMT_Q8_0), (oracle.FMT_Q4_0, oracle.FMT_Q4_0),
+           (oracle.FMT_Q4_0, oracle.FMT_Q8_0)]
+_QUANT = {oracle.FMT_Q8_0: oracle.quantize_q8_0, oracle.FMT_Q4_0: oracle.quantize_q4_0}
+_DEQ = {oracle.FMT_Q8_0: oracle.dequant_q8_0, oracle.FMT_Q4_0: oracle.dequant_q4_0}
+
+
+def _fmt_cache(H, D, cap, k_fmt, v_fmt, seed):
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((cap, H, D)).astype(np.float32)
+    v = rng.standard_normal((cap, H, D)).astype(np.float32)
+    k[:, :, :4] *= 8
+    kc, vc = oracle.empty_cache(H, D, cap, k_fmt=k_fmt, v_fmt=v_fmt)
+    oracle.append(kc, vc, k, v, 0)
+    return k, v, kc, vc
+
+
+@pytest.mark.parametrize("k_fmt,v_fmt", FORMATS)
+def test_format_append_writes_each_tensors_blocks(k_fmt, v_fmt):
+    H, D, cap = 2, 64, 5
+    k, v, kc, vc = _fmt_cache(H, D, cap, k_fmt, v_fmt, 11)
+    for h in range(H):
+        assert np.array_equal(kc[h].reshape(-1), _QUANT[k_fmt](k[:, h].reshape(-1)))
+        assert np.array_equal(vc[h].reshape(-1), _QUANT[v_fmt](v[:, h].reshape(-1)))
+
+
+@pytest.mark.parametrize("k_fmt,v_fmt", FORMATS)
+def test_format_single_key_and_brute_force(k_fmt, v_fmt):
+    H, D, Hq, T = 2, 64, 4, 2
+    n_kv = 9
+    k, v, kc, vc = _fmt_cache(H, D, n_kv, k_fmt, v_fmt, 12)
+    K = _DEQ[k_fmt](kc).reshape(H, n_kv, D)
+    V = _DEQ[v_fmt](vc).reshape(H, n_kv, D)
+    q = _q(T, Hq, D, 13)
+    # one key: its V row and its own score
+    out, lse = oracle.decode_attn(kc, vc, q[:1], n_kv=1, chunk=64, scale=SCALE)
+    for g in range(Hq):
+        h = g // (Hq // H)
+        assert np.array_equal(out[0, g, 0], V[h, 0])
+        assert abs(lse[0, g, 0] - SCALE * float(np.dot(q[0, g].astype(np.float64), K[h, 0]))) < 1e-12
+    # brute force over the dequantized rows, causal verify batch, one chunk
+    out, lse = oracle.decode_attn(kc, vc, q, n_kv=n_kv, chunk=64, scale=SCALE)
+    for t in range(T):
+        for g in range(Hq):
+            h = g // (Hq // H)
+            n = n_kv - T + t + 1
+            s = SCALE * (K[h, :n] @ q[t, g].astype(np.float64))
+            w = np.exp(s - s.max())
+            ref = (w / w.sum()) @ V[h, :n]
+            assert np.allclose(out[t, g, 0], ref, rtol=0, atol=1e-12)
+            assert abs(lse[t, g, 0] - (s.max() + math.log(w.sum()))) < 1e-12
