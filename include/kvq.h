@@ -50,6 +50,10 @@
  *     -> one head-row of a token is head_dim/32*34 bytes (272 B at 256)
  *  V: [n_kv_heads][capacity][head_dim/32] Q4_0 blocks
  *     -> one head-row is head_dim/32*18 bytes (144 B at 256)
+ *  That is the pages' configuration (kvq_layer k_type = v_type = 0).  Either
+ *  tensor may instead use the other format (KVQ_TYPE_Q8_0 / KVQ_TYPE_Q4_0,
+ *  the q8_0 and q4_0 choices of the KV-cache guide's levers section); its
+ *  head-rows are then head_dim/32 blocks of that format.
  *  Head-rows of consecutive tokens of a head are contiguous, so a run of
  *  tokens is one contiguous byte range.  Both base pointers must be 16-byte
  *  aligned and capacity a multiple of 8: then every head starts on a 16-byte
@@ -90,6 +94,19 @@ typedef void *kvq_stream;
 
 /* One attention layer of the cache.  All layers passed to one call must have
  * the same n_kv_heads and head_dim. */
+/* Block format of a cache tensor.  KVQ_TYPE_DEFAULT is Q8_0 for K and Q4_0
+ * for V.  All layers passed to one call must use the same formats.  Append,
+ * the general decode path (kvq_decode_attn, kvq_decode_step,
+ * kvq_decode_merged_static, kvq_stream_decode) accept every combination; the
+ * tiled decode kernel, the fused step's single launch and kvq_prefill_attn
+ * implement the default pair only (decode falls back to the general kernel,
+ * the step to three launches, prefill returns KVQ_ERR_UNSUPPORTED). */
+typedef enum kvq_type {
+    KVQ_TYPE_DEFAULT = 0,
+    KVQ_TYPE_Q8_0 = 1,   /* 34 B per 32 elements */
+    KVQ_TYPE_Q4_0 = 2    /* 18 B per 32 elements */
+} kvq_type;
+
 typedef struct kvq_layer {
     void *k;             /* K blocks, layout above (device memory, or pinned
                             host memory for kvq_stream_decode's host_layers) */
@@ -97,6 +114,8 @@ typedef struct kvq_layer {
     int64_t capacity;    /* tokens per head the two arrays hold              */
     int32_t n_kv_heads;  /* KV heads (4 in the pages' hybrid model)          */
     int32_t head_dim;    /* elements per head-row, a multiple of 32, <= 512  */
+    int32_t k_type;      /* kvq_type of K (0: Q8_0)                          */
+    int32_t v_type;      /* kvq_type of V (0: Q4_0)                          */
 } kvq_layer;
 
 /* Largest number of layers one call accepts (layer tables travel as kernel
@@ -126,7 +145,8 @@ kvq_status kvq_quantize_q8_0(const float *x, void *blocks, int64_t n, kvq_stream
 kvq_status kvq_quantize_q4_0(const float *x, void *blocks, int64_t n, kvq_stream stream);
 
 /* Quantize-on-append of new K/V rows into rows [pos, pos+n_tok) of every KV
- * head of n_layers layers (K -> Q8_0, V -> Q4_0).
+ * head of n_layers layers (K -> Q8_0, V -> Q4_0, or the layers' k_type /
+ * v_type).
  * Source: the KV-cache guide's levers section (the KV cache is stored
  * quantized); the Q8_0 K / Q4_0 V cache of the RX 9070 XT page.
  *  layers  host array of n_layers kvq_layer (device caches)
@@ -295,7 +315,8 @@ kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_layers,
                              kvq_stream copy);
 
 /* Adaptive residency: how many of n_layers layers (each n_kv_heads x capacity
- * K and V head-rows at head_dim) can stay resident in budget_bytes of device
+ * K and V head-rows at head_dim, in block formats k_type / v_type, 0 for the
+ * defaults) can stay resident in budget_bytes of device
  * memory while the rest stream through kvq_stream_decode's two slots of one
  * layer each.  n_layers if everything fits (no slots are needed then);
  * otherwise the largest R <= n_layers - 1 with (R + 2) layers <= budget; -1 if
@@ -303,7 +324,7 @@ kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_layers,
  * Source: "What shipped" / "Why it matters" of the ROCm streaming page (a
  * bounded working set streamed from host RAM when the cache does not fit). */
 int kvq_resident_layers(size_t budget_bytes, int n_layers, int64_t capacity, int n_kv_heads,
-                        int head_dim);
+                        int head_dim, int k_type, int v_type);
 
 /* ---------------------------------------------------------------------- */
 /* Decode + merge without caller-provided scratch                          */

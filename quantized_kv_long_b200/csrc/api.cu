@@ -76,6 +76,11 @@ static kvq_status check_layers(const kvq_layer *layers, int n_layers, const char
         return set_error(KVQ_ERR_UNSUPPORTED, "%s: head_dim=%d > 512", fn, D);
     for (int l = 0; l < n_layers; ++l) {
         const kvq_layer &L = layers[l];
+        for (const int t : {L.k_type, L.v_type})
+            if (t != KVQ_TYPE_DEFAULT && t != KVQ_TYPE_Q8_0 && t != KVQ_TYPE_Q4_0)
+                return set_error(KVQ_ERR_INVALID_ARG, "%s: layer %d has block type %d", fn, l, t);
+        if (k_type_of(L) != k_type_of(layers[0]) || v_type_of(L) != v_type_of(layers[0]))
+            return set_error(KVQ_ERR_INVALID_ARG, "%s: layer %d differs in block formats", fn, l);
         if (!L.k || !L.v)
             return set_error(KVQ_ERR_INVALID_ARG, "%s: layer %d has a NULL cache pointer", fn, l);
         if (L.n_kv_heads != H || L.head_dim != D)
@@ -162,6 +167,8 @@ static kvq_status fill_decode(const kvq_layer *layers, int n_layers, const uint1
     a.head_dim = layers[0].head_dim;
     a.n_q_heads = n_q_heads;
     a.T = T;
+    a.k_type = k_type_of(layers[0]);
+    a.v_type = v_type_of(layers[0]);
     a.n_kv = n_kv;
     a.chunk = chunk;
     a.scale = scale;
@@ -268,7 +275,8 @@ kvq_status kvq_append(const kvq_layer *layers, int n_layers, const float *k_new,
         t.v[l] = l < n_layers ? static_cast<uint8_t *>(layers[l].v) : nullptr;
         t.cap[l] = l < n_layers ? layers[l].capacity : 0;
     }
-    launch_append(t, n_layers, H, D, k_new, v_new, pos, n_tok, as_stream(stream));
+    launch_append(t, n_layers, H, D, k_type_of(layers[0]), v_type_of(layers[0]), k_new, v_new,
+                  pos, n_tok, as_stream(stream));
     return check_launch(fn);
 }
 
@@ -377,6 +385,8 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
     if (!prefill_supported(n_q_heads, H, D))
         return set_error(KVQ_ERR_UNSUPPORTED, "%s: head_dim=%d, group=%d not supported", fn, D,
                          n_q_heads / H);
+    if (k_type_of(layers[0]) != KVQ_TYPE_Q8_0 || v_type_of(layers[0]) != KVQ_TYPE_Q4_0)
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: only Q8_0 K with Q4_0 V is implemented", fn);
     const size_t ws = prefill_workspace_bytes(n_layers, n_q_heads, H, T, D);
     if (ws > 0 && (workspace == nullptr || ws_bytes < ws))
         return set_error(KVQ_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn,

@@ -16,6 +16,12 @@ constexpr int Q4_0_BYTES = 18;   // fp16 d + 16 bytes of nibbles
 __host__ __device__ inline int64_t k_row_bytes(int head_dim) { return (int64_t)(head_dim / QK) * Q8_0_BYTES; }
 __host__ __device__ inline int64_t v_row_bytes(int head_dim) { return (int64_t)(head_dim / QK) * Q4_0_BYTES; }
 
+// Block formats (kvq_type resolved: KVQ_TYPE_DEFAULT becomes Q8_0 for K, Q4_0 for V).
+__host__ __device__ inline int block_bytes(int type) { return type == KVQ_TYPE_Q8_0 ? Q8_0_BYTES : Q4_0_BYTES; }
+__host__ __device__ inline int64_t row_bytes(int type, int head_dim) { return (int64_t)(head_dim / QK) * block_bytes(type); }
+inline int k_type_of(const kvq_layer &l) { return l.k_type ? l.k_type : KVQ_TYPE_Q8_0; }
+inline int v_type_of(const kvq_layer &l) { return l.v_type ? l.v_type : KVQ_TYPE_Q4_0; }
+
 // Layer table passed by value as a kernel parameter.
 struct LayerTable {
     const uint8_t *k[KVQ_MAX_LAYERS];
@@ -53,14 +59,15 @@ inline cudaStream_t as_stream(kvq_stream s) { return reinterpret_cast<cudaStream
 void launch_quantize_q8_0(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s);
 void launch_quantize_q4_0(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s);
 void launch_append(const MutLayerTable &t, int n_layers, int n_kv_heads, int head_dim,
-                   const float *k_new, const float *v_new, int64_t pos, int n_tok,
-                   cudaStream_t s);
+                   int k_type, int v_type, const float *k_new, const float *v_new, int64_t pos,
+                   int n_tok, cudaStream_t s);
 void launch_merge_lse(const float *out_part, const float *lse_part, int64_t rows, int n_chunks,
                       int head_dim, float *out, float *lse, cudaStream_t s);
 
 struct DecodeArgs {
     LayerTable layers;
     int n_layers, n_kv_heads, head_dim, n_q_heads, T;
+    int k_type, v_type;  // resolved block formats (KVQ_TYPE_Q8_0 / KVQ_TYPE_Q4_0)
     int64_t n_kv;
     int chunk;
     float scale;

@@ -602,7 +602,8 @@ bool launch_tc(const DecodeArgs &a, cudaStream_t s)
 bool decode_tc_supported(const DecodeArgs &a)
 {
     const int rows = (a.n_q_heads / a.n_kv_heads) * a.T;
-    return a.head_dim == 256 && rows <= 24;
+    return a.head_dim == 256 && rows <= 24 && a.k_type == KVQ_TYPE_Q8_0 &&
+           a.v_type == KVQ_TYPE_Q4_0;
 }
 
 bool launch_decode(const DecodeArgs &a, cudaStream_t s)

@@ -13,6 +13,9 @@
 // the OSCAR2 page: the max covers complete scores; GQA section of the KV-cache
 // guide): row r = t*G + g is query head h*G + g of token t and sees keys
 // j <= n_kv - T + t of chunk c = keys [c*chunk, (c+1)*chunk).
+//
+// K and V may each be in either block format (template parameters KT, VT:
+// KVQ_TYPE_Q8_0 or KVQ_TYPE_Q4_0); the pages' configuration is Q8_0 K / Q4_0 V.
 #include "common.cuh"
 
 namespace kvq {
@@ -20,6 +23,23 @@ namespace kvq {
 constexpr int SIMPLE_THREADS = 256;
 constexpr int SIMPLE_TILE = 64;
 
+// Integer value of element i (0..31) of a block: int8 q (Q8_0) or nibble - 8
+// (Q4_0: byte i holds element i in the low nibble and element i + 16 in the high).
+template <int TYPE>
+__device__ __forceinline__ int block_int(const uint8_t *blk, int i)
+{
+    if (TYPE == KVQ_TYPE_Q8_0)
+        return (int)(int8_t)blk[2 + i];
+    const uint8_t byte = blk[2 + (i & 15)];
+    return (i < 16 ? (byte & 15) : (byte >> 4)) - 8;
+}
+
+__device__ __forceinline__ float block_d(const uint8_t *blk)
+{
+    return __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
+}
+
+template <int KT, int VT>
 __global__ void __launch_bounds__(SIMPLE_THREADS)
 decode_simple_kernel(DecodeArgs a)
 {
@@ -39,8 +59,9 @@ decode_simple_kernel(DecodeArgs a)
     const int n_chunks = (int)((a.n_kv + a.chunk - 1) / a.chunk);
     const int64_t c0 = (int64_t)c * a.chunk;
     const int64_t c1 = c0 + a.chunk < a.n_kv ? c0 + a.chunk : a.n_kv;
-    const uint8_t *kb = a.layers.k[layer] + (int64_t)h * a.layers.cap[layer] * k_row_bytes(D);
-    const uint8_t *vb = a.layers.v[layer] + (int64_t)h * a.layers.cap[layer] * v_row_bytes(D);
+    const int64_t krow = row_bytes(KT, D), vrow = row_bytes(VT, D);
+    const uint8_t *kb = a.layers.k[layer] + (int64_t)h * a.layers.cap[layer] * krow;
+    const uint8_t *vb = a.layers.v[layer] + (int64_t)h * a.layers.cap[layer] * vrow;
 
     for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
         const int r = p / D, i = p % D;
@@ -62,16 +83,15 @@ decode_simple_kernel(DecodeArgs a)
             const int t = r / G;
             float s = -INFINITY;
             if (j < c1 && j <= a.n_kv - a.T + t) {
-                const uint8_t *kr = kb + j * k_row_bytes(D);
+                const uint8_t *kr = kb + j * krow;
                 const float *qr = q_s + r * D;
                 float tot = 0.0f;
                 for (int b = 0; b < nb; ++b) {
-                    const uint8_t *blk = kr + b * Q8_0_BYTES;
-                    const float d = __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
+                    const uint8_t *blk = kr + b * block_bytes(KT);
                     float part = 0.0f;
                     for (int i = 0; i < QK; ++i)
-                        part += qr[b * QK + i] * (float)(int8_t)blk[2 + i];
-                    tot += d * part;
+                        part += qr[b * QK + i] * (float)block_int<KT>(blk, i);
+                    tot += block_d(blk) * part;
                 }
                 s = a.scale * tot;
             }
@@ -112,11 +132,8 @@ decode_simple_kernel(DecodeArgs a)
                 const float pw = p_s[r * SIMPLE_TILE + jj];
                 if (pw == 0.0f)
                     continue;
-                const uint8_t *blk = vb + (j0 + jj) * v_row_bytes(D) + b * Q4_0_BYTES;
-                const float d = __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
-                const uint8_t byte = blk[2 + (ii & 15)];
-                const int u = ii < 16 ? (byte & 15) : (byte >> 4);
-                o += pw * (d * (float)(u - 8));
+                const uint8_t *blk = vb + (j0 + jj) * vrow + b * block_bytes(VT);
+                o += pw * (block_d(blk) * (float)block_int<VT>(blk, ii));
             }
             acc[p] = o;
         }
@@ -139,6 +156,19 @@ size_t decode_simple_smem(int R, int D)
     return sizeof(float) * ((size_t)2 * R * D + (size_t)R * SIMPLE_TILE + 3 * (size_t)R);
 }
 
+template <int KT, int VT>
+static bool launch_simple_typed(const DecodeArgs &a, size_t smem, cudaStream_t s)
+{
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(decode_simple_kernel<KT, VT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return false;
+    const int n_chunks = (int)((a.n_kv + a.chunk - 1) / a.chunk);
+    dim3 grid(n_chunks, a.n_kv_heads, a.n_layers);
+    decode_simple_kernel<KT, VT><<<grid, SIMPLE_THREADS, smem, s>>>(a);
+    return true;
+}
+
 bool launch_decode_simple(const DecodeArgs &a, cudaStream_t s)
 {
     const int G = a.n_q_heads / a.n_kv_heads;
@@ -146,14 +176,16 @@ bool launch_decode_simple(const DecodeArgs &a, cudaStream_t s)
     const size_t smem = decode_simple_smem(R, a.head_dim);
     if (smem > 227 * 1024)
         return false;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(decode_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return false;
-    const int n_chunks = (int)((a.n_kv + a.chunk - 1) / a.chunk);
-    dim3 grid(n_chunks, a.n_kv_heads, a.n_layers);
-    decode_simple_kernel<<<grid, SIMPLE_THREADS, smem, s>>>(a);
-    return true;
+    constexpr int Q8 = KVQ_TYPE_Q8_0, Q4 = KVQ_TYPE_Q4_0;
+    if (a.k_type == Q8 && a.v_type == Q4)
+        return launch_simple_typed<Q8, Q4>(a, smem, s);
+    if (a.k_type == Q8 && a.v_type == Q8)
+        return launch_simple_typed<Q8, Q8>(a, smem, s);
+    if (a.k_type == Q4 && a.v_type == Q4)
+        return launch_simple_typed<Q4, Q4>(a, smem, s);
+    if (a.k_type == Q4 && a.v_type == Q8)
+        return launch_simple_typed<Q4, Q8>(a, smem, s);
+    return false;
 }
 
 }  // namespace kvq

@@ -58,10 +58,11 @@ void launch_quantize_q4_0(const float *x, uint8_t *blocks, int64_t n, cudaStream
 }
 
 // Append: one CTA per (layer, token, kv head); warps [0, nb) quantize the K
-// blocks of the head-row, warps [nb, 2 nb) the V blocks (nb = head_dim / 32).
-__global__ void append_kernel(MutLayerTable t, int n_kv_heads, int head_dim,
-                              const float *__restrict__ k_new, const float *__restrict__ v_new,
-                              int64_t pos, int n_tok)
+// blocks of the head-row, warps [nb, 2 nb) the V blocks (nb = head_dim / 32),
+// each tensor in its block format.
+__global__ void append_kernel(MutLayerTable t, int n_kv_heads, int head_dim, int k_type,
+                              int v_type, const float *__restrict__ k_new,
+                              const float *__restrict__ v_new, int64_t pos, int n_tok)
 {
     const int h = blockIdx.x % n_kv_heads;
     const int tok = (blockIdx.x / n_kv_heads) % n_tok;
@@ -72,24 +73,25 @@ __global__ void append_kernel(MutLayerTable t, int n_kv_heads, int head_dim,
     const int b = is_v ? w - nb : w;
     const size_t src = (((size_t)layer * n_tok + tok) * n_kv_heads + h) * head_dim + (size_t)b * QK;
     const int64_t row = (int64_t)h * t.cap[layer] + pos + tok;
-    if (!is_v) {
-        uint8_t *dst = t.k[layer] + row * k_row_bytes(head_dim) + (int64_t)b * Q8_0_BYTES;
-        warp_quant_q8_0(k_new[src + lane], dst, lane);
-    } else {
-        uint8_t *dst = t.v[layer] + row * v_row_bytes(head_dim) + (int64_t)b * Q4_0_BYTES;
-        warp_quant_q4_0(v_new[src + lane], dst, lane);
-    }
+    const int type = is_v ? v_type : k_type;  // uniform across the warp
+    uint8_t *dst = (is_v ? t.v[layer] : t.k[layer]) + row * row_bytes(type, head_dim) +
+                   (int64_t)b * block_bytes(type);
+    const float x = (is_v ? v_new : k_new)[src + lane];
+    if (type == KVQ_TYPE_Q8_0)
+        warp_quant_q8_0(x, dst, lane);
+    else
+        warp_quant_q4_0(x, dst, lane);
 }
 
 void launch_append(const MutLayerTable &t, int n_layers, int n_kv_heads, int head_dim,
-                   const float *k_new, const float *v_new, int64_t pos, int n_tok,
-                   cudaStream_t s)
+                   int k_type, int v_type, const float *k_new, const float *v_new, int64_t pos,
+                   int n_tok, cudaStream_t s)
 {
     const int64_t ctas = (int64_t)n_layers * n_tok * n_kv_heads;
     const int threads = 2 * (head_dim / QK) * 32;
     // grid.x is at most 2^31-1; n_tok is an int and n_layers <= 64, heads small
-    append_kernel<<<(unsigned)ctas, threads, 0, s>>>(t, n_kv_heads, head_dim, k_new, v_new, pos,
-                                                     n_tok);
+    append_kernel<<<(unsigned)ctas, threads, 0, s>>>(t, n_kv_heads, head_dim, k_type, v_type,
+                                                     k_new, v_new, pos, n_tok);
 }
 
 }  // namespace kvq

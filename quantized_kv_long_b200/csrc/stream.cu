@@ -126,9 +126,11 @@ extern "C" kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_laye
                              lse_part, fn);
         if (st != KVQ_OK)
             return st;
-        if (dev_slots[0].n_kv_heads != H || dev_slots[0].head_dim != D)
-            return set_error(KVQ_ERR_INVALID_ARG, "%s: slots and host layers differ in shape",
-                             fn);
+        if (dev_slots[0].n_kv_heads != H || dev_slots[0].head_dim != D ||
+            k_type_of(dev_slots[0]) != k_type_of(host_layers[0]) ||
+            v_type_of(dev_slots[0]) != v_type_of(host_layers[0]))
+            return set_error(KVQ_ERR_INVALID_ARG,
+                             "%s: slots and host layers differ in shape or block formats", fn);
         for (int s = 0; s < 2; ++s)
             if (placement(dev_slots[s].k) != 2 || placement(dev_slots[s].v) != 2)
                 return set_error(KVQ_ERR_INVALID_ARG,
@@ -143,7 +145,8 @@ extern "C" kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_laye
     if (cudaEventRecord(start, cs) != cudaSuccess || cudaStreamWaitEvent(ps, start, 0) != cudaSuccess)
         return set_error(KVQ_ERR_CUDA, "%s: event ordering failed", fn);
 
-    const int64_t kr = k_row_bytes(D), vr = v_row_bytes(D);
+    const int64_t kr = row_bytes(k_type_of(host_layers[0]), D);
+    const int64_t vr = row_bytes(v_type_of(host_layers[0]), D);
     const int fail_at = fail_copy_layer();
     int i_streamed = 0;  // streamed layers enqueued so far
     for (int L = 0; L < n_layers; ++L) {
@@ -196,12 +199,16 @@ extern "C" kvq_status kvq_stream_decode(const kvq_layer *host_layers, int n_laye
 }
 
 extern "C" int kvq_resident_layers(size_t budget_bytes, int n_layers, int64_t capacity,
-                                   int n_kv_heads, int head_dim)
+                                   int n_kv_heads, int head_dim, int k_type, int v_type)
 {
     if (n_layers < 1 || capacity < 1 || n_kv_heads < 1 || head_dim < QK || head_dim % QK != 0)
         return -1;
+    for (const int t : {k_type, v_type})
+        if (t != KVQ_TYPE_DEFAULT && t != KVQ_TYPE_Q8_0 && t != KVQ_TYPE_Q4_0)
+            return -1;
+    const int kt = k_type ? k_type : KVQ_TYPE_Q8_0, vt = v_type ? v_type : KVQ_TYPE_Q4_0;
     const double layer = (double)n_kv_heads * (double)capacity *
-                         (double)(k_row_bytes(head_dim) + v_row_bytes(head_dim));
+                         (double)(row_bytes(kt, head_dim) + row_bytes(vt, head_dim));
     const double budget = (double)budget_bytes;
     if (layer * n_layers <= budget)
         return n_layers;  // everything resident: no slots needed

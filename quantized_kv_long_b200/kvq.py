@@ -42,11 +42,20 @@ KVQ_MAX_DECODE_T = 4
 KVQ_STATIC_SCRATCH_BYTES = 8 << 20
 
 QK, Q8_0_BYTES, Q4_0_BYTES = 32, 34, 18
+KVQ_TYPE_DEFAULT, KVQ_TYPE_Q8_0, KVQ_TYPE_Q4_0 = 0, 1, 2
+
+
+def block_bytes(kvq_type: int, tensor: str) -> int:
+    """Bytes per 32-element block of a cache tensor ('k' or 'v') in ``kvq_type``."""
+    if kvq_type == KVQ_TYPE_DEFAULT:
+        kvq_type = KVQ_TYPE_Q8_0 if tensor == "k" else KVQ_TYPE_Q4_0
+    return Q8_0_BYTES if kvq_type == KVQ_TYPE_Q8_0 else Q4_0_BYTES
 
 
 class kvq_layer(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("capacity", ctypes.c_int64),
-                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("k_type", ctypes.c_int32), ("v_type", ctypes.c_int32)]
 
 
 class KvqError(RuntimeError):
@@ -72,7 +81,7 @@ _SIGS = {
                            _P], _I32),
     "kvq_decode_merged_static": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P],
                                  _I32),
-    "kvq_resident_layers": ([_SZ, _I32, _I64, _I32, _I32], _I32),
+    "kvq_resident_layers": ([_SZ, _I32, _I64, _I32, _I32, _I32, _I32], _I32),
     "kvq_workspace_bytes": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "kvq_check": ([_P], _I32),
     "kvq_status_string": ([_I32], ctypes.c_char_p),
@@ -205,8 +214,9 @@ def kvq_decode_merged_static(layers, q, n_q_heads: int, T: int, n_kv: int, chunk
 
 
 def kvq_resident_layers(budget_bytes: int, n_layers: int, capacity: int, n_kv_heads: int,
-                        head_dim: int) -> int:
-    return _lib.kvq_resident_layers(budget_bytes, n_layers, capacity, n_kv_heads, head_dim)
+                        head_dim: int, k_type: int = 0, v_type: int = 0) -> int:
+    return _lib.kvq_resident_layers(budget_bytes, n_layers, capacity, n_kv_heads, head_dim,
+                                    k_type, v_type)
 
 
 def kvq_workspace_bytes(op: int, n_layers: int, n_q_heads: int, n_kv_heads: int, T: int,
@@ -222,17 +232,22 @@ class QuantizedKVCache:
     """Caller-owned cache memory in the library's layout (torch allocates it).
 
     K of layer ``l``: uint8 ``[n_kv_heads, capacity, head_dim // 32 * 34]``;
-    V: ``[n_kv_heads, capacity, head_dim // 32 * 18]``.  ``device="cpu"`` with
-    ``pin=True`` gives pinned host memory for :func:`kvq_stream_decode`.
+    V: ``[n_kv_heads, capacity, head_dim // 32 * 18]`` (the default Q8_0 K /
+    Q4_0 V; ``k_type`` / ``v_type`` select the other block format per tensor).
+    ``device="cpu"`` with ``pin=True`` gives pinned host memory for
+    :func:`kvq_stream_decode`.
     """
 
     def __init__(self, n_layers: int, n_kv_heads: int, head_dim: int, capacity: int,
-                 device="cuda", pin: bool = False):
+                 device="cuda", pin: bool = False, k_type: int = KVQ_TYPE_DEFAULT,
+                 v_type: int = KVQ_TYPE_DEFAULT):
         if capacity % 8:
             raise ValueError("capacity must be a multiple of 8")
         self.n_layers, self.n_kv_heads, self.head_dim, self.capacity = (
             n_layers, n_kv_heads, head_dim, capacity)
-        kb, vb = head_dim // QK * Q8_0_BYTES, head_dim // QK * Q4_0_BYTES
+        self.k_type, self.v_type = k_type, v_type
+        kb = head_dim // QK * block_bytes(k_type, "k")
+        vb = head_dim // QK * block_bytes(v_type, "v")
         kw = dict(dtype=torch.uint8, device=device)
         if pin:
             kw["pin_memory"] = True
@@ -241,7 +256,7 @@ class QuantizedKVCache:
 
     def layer(self, l: int) -> kvq_layer:
         return kvq_layer(self.k[l].data_ptr(), self.v[l].data_ptr(), self.capacity,
-                         self.n_kv_heads, self.head_dim)
+                         self.n_kv_heads, self.head_dim, self.k_type, self.v_type)
 
     def layers(self, start: int = 0, stop: int | None = None) -> list[kvq_layer]:
         stop = self.n_layers if stop is None else stop
@@ -253,6 +268,7 @@ class QuantizedKVCache:
 
 
 def make_layers(ks: Sequence[torch.Tensor], vs: Sequence[torch.Tensor], capacity: int,
-                n_kv_heads: int, head_dim: int) -> list[kvq_layer]:
-    return [kvq_layer(k.data_ptr(), v.data_ptr(), capacity, n_kv_heads, head_dim)
+                n_kv_heads: int, head_dim: int, k_type: int = KVQ_TYPE_DEFAULT,
+                v_type: int = KVQ_TYPE_DEFAULT) -> list[kvq_layer]:
+    return [kvq_layer(k.data_ptr(), v.data_ptr(), capacity, n_kv_heads, head_dim, k_type, v_type)
             for k, v in zip(ks, vs)]

@@ -35,11 +35,21 @@ def assert_attn_close(out, lse, ref_out, ref_lse, what=""):
         assert lerr <= LSE_RTOL, f"{what}: lse relative error {lerr:.3e} > {LSE_RTOL}"
 
 
-def fill_both(w: wl.Workload, layers, n_rows: int, capacity: int, device="cuda"):
+def oracle_fmt(kvq, kvq_type: int, tensor: str) -> int:
+    """The oracle's block format for a kvq_type of a cache tensor ('k' or 'v')."""
+    if kvq_type == kvq.KVQ_TYPE_DEFAULT:
+        return oracle.FMT_Q8_0 if tensor == "k" else oracle.FMT_Q4_0
+    return {kvq.KVQ_TYPE_Q8_0: oracle.FMT_Q8_0, kvq.KVQ_TYPE_Q4_0: oracle.FMT_Q4_0}[kvq_type]
+
+
+def fill_both(w: wl.Workload, layers, n_rows: int, capacity: int, device="cuda", k_type=0,
+              v_type=0):
     """Quantize rows [0, n_rows) of the given layers on the GPU (through
-    kvq_append) and on the CPU (oracle).  Returns (gpu cache, oracle caches)."""
+    kvq_append) and on the CPU (oracle), K and V in the given block formats
+    (0 = the default Q8_0 K / Q4_0 V).  Returns (gpu cache, oracle caches)."""
     from quantized_kv_long_b200 import kvq
-    cache = kvq.QuantizedKVCache(len(layers), w.n_kv_heads, w.head_dim, capacity, device=device)
+    cache = kvq.QuantizedKVCache(len(layers), w.n_kv_heads, w.head_dim, capacity, device=device,
+                                 k_type=k_type, v_type=v_type)
     orc = []
     for i, l in enumerate(layers):
         k = wl.kv_rows(w, l, 0, 0, n_rows)
@@ -47,7 +57,9 @@ def fill_both(w: wl.Workload, layers, n_rows: int, capacity: int, device="cuda")
         kt = torch.from_numpy(k).to(device)
         vt = torch.from_numpy(v).to(device)
         kvq.kvq_append(cache.layer(i), kt, vt, 0, n_rows)
-        kc, vc = oracle.empty_cache(w.n_kv_heads, w.head_dim, capacity)
+        kc, vc = oracle.empty_cache(w.n_kv_heads, w.head_dim, capacity,
+                                    k_fmt=oracle_fmt(kvq, k_type, "k"),
+                                    v_fmt=oracle_fmt(kvq, v_type, "v"))
         oracle.append(kc, vc, k, v, 0)
         orc.append((kc, vc))
     torch.cuda.synchronize()

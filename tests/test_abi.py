@@ -51,9 +51,10 @@ A = 1 << 20  # a 16-byte aligned fake device address: never dereferenced here
 
 
 def _layer(kvq, **kw):
-    d = dict(k=A, v=A, capacity=1024, n_kv_heads=4, head_dim=256)
+    d = dict(k=A, v=A, capacity=1024, n_kv_heads=4, head_dim=256, k_type=0, v_type=0)
     d.update(kw)
-    return kvq.kvq_layer(d["k"], d["v"], d["capacity"], d["n_kv_heads"], d["head_dim"])
+    return kvq.kvq_layer(d["k"], d["v"], d["capacity"], d["n_kv_heads"], d["head_dim"],
+                         d["k_type"], d["v_type"])
 
 
 def test_quantize_validation(kvq):
@@ -190,3 +191,22 @@ def test_resident_layers_plan(kvq):
     assert plan(10**15, 1) == 1
     assert kvq.kvq_resident_layers(1 << 40, 0, 1024, 4, 256) == -1
     assert kvq.kvq_resident_layers(1 << 40, 4, 1024, 4, 48) == -1
+
+
+def test_block_format_validation(kvq):
+    """Block formats: unknown types and layers that differ are refused; prefill
+    implements the default pair only; the residency plan sizes layers by format."""
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, _layer(kvq, k_type=3), A, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, _layer(kvq, v_type=-1), A, A, 0, 1, 0)
+    # explicit Q8_0 K / Q4_0 V equals the default pair, so these two layers agree
+    mixed_ok = [_layer(kvq), _layer(kvq, k_type=kvq.KVQ_TYPE_Q8_0, v_type=kvq.KVQ_TYPE_Q4_0)]
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, mixed_ok + [_layer(kvq, v_type=1)],
+            A, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_decode_attn,
+            [_layer(kvq, k_type=2), _layer(kvq)], A, 24, 1, 1024, 256, 1 / 16, A, A, 0)
+    _raises(kvq, kvq.KVQ_ERR_UNSUPPORTED, kvq.kvq_prefill_attn, _layer(kvq, v_type=1, capacity=4096),
+            A, 24, 128, 1024, 1024, 1 / 16, A, A)
+    q8 = 4 * 262144 * (272 + 272)
+    assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 1, 1) == 3
+    assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 0, 0) == 4
+    assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 7, 0) == -1
