@@ -68,7 +68,6 @@ constexpr int TILE_H = BN * HD * 2;  // one f16 tile of 32 keys x 256 dims: 16 K
 constexpr int NR = 4;  // raw staging slots (bulk copies in flight ahead of the dequant)
 constexpr int NB = 3;  // f16 K^hi / K^lo / V^ tile slots
 constexpr int NS = 4;  // S / P slots in tensor memory
-constexpr int LA = 1;  // the PV of tile j - LA is issued after the QK^T of tile j
 constexpr int N_SOFT = 4, N_DEQ = 8;
 constexpr int W_PROD = N_SOFT + N_DEQ, W_MMA = W_PROD + 1;
 constexpr int PF_THREADS = (W_MMA + 1) * 32;  // 14 warps
@@ -83,6 +82,11 @@ constexpr uint32_t COL_O = 0, COL_Q = 256, COL_S0 = 384;
 static_assert(COL_S0 + NS * BN <= 512, "tensor-memory columns");
 static_assert(BN * 8 == N_DEQ * 32, "one K unit and one V unit per dequant thread and tile");
 static_assert(NB <= NS, "a K^ slot is reused only after the QK^T that read it");
+// The MMA warp waits only for k_full(j) and p_full(j - 1) per tile.  k_full(j)
+// completes after every dequant warp has finished V^ of tile j - 1 (program order
+// in each warp), which in turn waited for the PV of tile j - 1 - NB = j - NS to
+// finish; so k_full(j) also covers v_full(j - 1) and the S/P slot of tile j.
+static_assert(NS == NB + 1, "k_full(j) must imply that the PV of tile j - NS is done");
 
 struct PfSmemHead {
     uint64_t raw_full[NR], raw_free[NR], k_full[NB], v_full[NB], s_full[NS], p_full[NS],
@@ -509,9 +513,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         const uint64_t dv0 = ptx::smem_desc_sw128(smem + OFF_VH, BN * 128, 1024);
         int committed = -1;  // last tile whose PV was committed
         bool ok = wwait(&hd.q_ready, 0);
+        // PV of tile jj, issued after the QK^T of tile jj + 1: V^ is ready once
+        // k_full(jj + 1) has completed (see NS above); the last tile has no successor
+        // and waits for v_full itself
         auto issue_pv = [&](int jj) -> bool {
             const int vb = slot(jj, NB), sb = slot(jj, NS);
-            if (!wwait(&hd.v_full[vb], par(jj, NB)) || !wwait(&hd.p_full[sb], par(jj, NS)))
+            if ((jj == ntiles - 1 && !wwait(&hd.v_full[vb], par(jj, NB))) ||
+                !wwait(&hd.p_full[sb], par(jj, NS)))
                 return false;
             ptx::tc_fence_after();
             if (leader) {
@@ -528,9 +536,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         };
         for (int j = 0; ok && j < ntiles; ++j) {
             const int kb = slot(j, NB), sb = slot(j, NS);
-            // K^ of tile j is ready; S slot sb (P of tile j - NS) is free once that PV is done
-            ok = wwait(&hd.k_full[kb], par(j, NB)) &&
-                 (j < NS || wwait(&hd.pv_done[sb], par(j - NS, NS)));
+            // K^ of tile j is ready, and (see NS above) the PV of tile j - NS that read
+            // S/P slot sb is done
+            ok = wwait(&hd.k_full[kb], par(j, NB));
             if (!ok)
                 break;
             ptx::tc_fence_after();
@@ -548,11 +556,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
                 ptx::umma_commit(&hd.s_full[sb]);
             }
             __syncwarp();
-            if (j >= LA)
-                ok = issue_pv(j - LA);
+            if (j >= 1)
+                ok = issue_pv(j - 1);
         }
-        for (int jj = (ntiles > LA ? ntiles - LA : 0); ok && jj < ntiles; ++jj)
-            ok = issue_pv(jj);
+        if (ok)
+            ok = issue_pv(ntiles - 1);
         if (!ok && lane == 0)
             fail();
         // every committed MMA has finished before TMEM is freed (a commit tracks all
