@@ -267,9 +267,19 @@ kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k
  *  out, lse  device fp32 [n_layers][T][n_q_heads][head_dim] and [...][n_q_heads]
  *  page_out, page_lse  must be NULL: per-page partial outputs are not built
  *            (both set -> KVQ_ERR_UNSUPPORTED)
- *  workspace unused (kvq_workspace_bytes(KVQ_OP_PREFILL, ...) is 0); may be NULL
- * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (group size > 32, page outputs),
- *         CUDA. */
+ *  workspace optional, device, 256-B aligned.  NULL: each CTA of the
+ *            tensor-core path dequantizes the key tiles it reads.  Otherwise
+ *            ws_bytes >= kvq_prefill_workspace_bytes(n_layers, n_kv_heads,
+ *            head_dim, n_cached + T) and the call first expands every key tile
+ *            once into the workspace (f16 K^hi, K^lo, V^: 1,536 B per key and KV
+ *            head at head_dim 256), which the tensor-core kernel then copies in
+ *            without dequantizing (every row tile of a KV head reads the same
+ *            keys).  Same results bit for bit.  Ignored when the tensor-core
+ *            path does not run.  Owned by the caller; not used after the call's
+ *            work completes.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (group size > 32, page outputs,
+ *         block formats other than Q8_0 K / Q4_0 V), WORKSPACE (a workspace
+ *         smaller than needed), CUDA. */
 kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
                             int n_q_heads, int T, int64_t n_cached, int page, float scale,
                             float *out, float *lse, float *page_out, float *page_lse,
@@ -362,6 +372,11 @@ kvq_status kvq_decode_merged_static(const kvq_layer *layers, int n_layers, const
 /* ---------------------------------------------------------------------- */
 /* Housekeeping                                                            */
 /* ---------------------------------------------------------------------- */
+
+/* Bytes of the optional kvq_prefill_attn workspace for n_keys = n_cached + T
+ * keys: n_layers * n_kv_heads * ceil(n_keys / 32) * 49,152 at head_dim 256;
+ * 0 when the shape has no tensor-core path (head_dim != 256). */
+size_t kvq_prefill_workspace_bytes(int n_layers, int n_kv_heads, int head_dim, int64_t n_keys);
 
 #define KVQ_OP_DECODE 1
 #define KVQ_OP_PREFILL 2

@@ -408,11 +408,29 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
     a.lse = lse;
     a.page_out = page_out;
     a.page_lse = page_lse;
-    a.workspace = workspace;
-    a.ws_bytes = ws_bytes;
+    // optional workspace: the f16 key tiles of the tensor-core path, expanded once
+    a.workspace = nullptr;
+    a.ws_bytes = 0;
+    const size_t exp = prefill_expand_bytes(n_layers, H, D, n_cached + T);
+    if (workspace != nullptr && exp > 0) {
+        if (ws_bytes < exp)
+            return set_error(KVQ_ERR_WORKSPACE,
+                             "%s: workspace of %zu bytes given, the expanded tiles need %zu "
+                             "(kvq_prefill_workspace_bytes); pass NULL to dequantize in place",
+                             fn, ws_bytes, exp);
+        if (!aligned(workspace, 256))
+            return set_error(KVQ_ERR_ALIGNMENT, "%s: workspace not 256-byte aligned", fn);
+        a.workspace = workspace;
+        a.ws_bytes = ws_bytes;
+    }
     KVQ_TRY(status_word(&a.status));
     launch_prefill(a, as_stream(stream));
     return check_launch(fn);
+}
+
+size_t kvq_prefill_workspace_bytes(int n_layers, int n_kv_heads, int head_dim, int64_t n_keys)
+{
+    return prefill_expand_bytes(n_layers, n_kv_heads, head_dim, n_keys);
 }
 
 size_t kvq_workspace_bytes(int op, int n_layers, int n_q_heads, int n_kv_heads, int T,

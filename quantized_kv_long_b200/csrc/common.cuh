@@ -101,6 +101,9 @@ struct PrefillArgs {
     unsigned int *status;
 };
 size_t prefill_workspace_bytes(int n_layers, int n_q_heads, int n_kv_heads, int T, int head_dim);
+// Optional workspace of the tensor-core path: the f16 key tiles expanded once per
+// call (0 if the shape has no such path).  n_keys = n_cached + T.
+size_t prefill_expand_bytes(int n_layers, int n_kv_heads, int head_dim, int64_t n_keys);
 bool prefill_supported(int n_q_heads, int n_kv_heads, int head_dim);
 void launch_prefill(const PrefillArgs &a, cudaStream_t s);
 

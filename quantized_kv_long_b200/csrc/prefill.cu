@@ -69,8 +69,13 @@ constexpr int NR = 4;  // raw staging slots (bulk copies in flight ahead of the 
 constexpr int NB = 3;  // f16 K^hi / K^lo / V^ tile slots
 constexpr int NS = 4;  // S / P slots in tensor memory
 constexpr int N_SOFT = 4, N_DEQ = 8;
-constexpr int W_PROD = N_SOFT + N_DEQ, W_MMA = W_PROD + 1;
-constexpr int PF_THREADS = (W_MMA + 1) * 32;  // 14 warps
+// roles: softmax warps, dequant warps (none when the f16 tiles were expanded into
+// the workspace beforehand), the producer warp, the MMA warp
+template <bool PRE> constexpr int n_deq() { return PRE ? 0 : N_DEQ; }
+template <bool PRE> constexpr int w_prod() { return N_SOFT + n_deq<PRE>(); }
+template <bool PRE> constexpr int w_mma() { return w_prod<PRE>() + 1; }
+template <bool PRE> constexpr int pf_threads() { return (w_mma<PRE>() + 1) * 32; }  // 14 / 6 warps
+constexpr int TILE3 = 3 * TILE_H;  // one key tile's K^hi, K^lo, V^ in the workspace: 48 KB
 constexpr uint64_t WAIT_NS = 1000000000ull;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
@@ -153,7 +158,97 @@ __device__ __forceinline__ void sts128(uint8_t *p, uint32_t a, uint32_t b, uint3
     *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
 }
 
-__global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const PrefillArgs a, int row0)
+// Dequant of one (key r, 32-element block bk) unit of a raw tile into the f16
+// tiles (offsets off[m4] of dims 32 bk + 8 m4 of key r, from sw_off); keys past
+// the end (in = false) are written as zeros so that 0-weight products stay 0.
+// K: rk = raw Q8_0 head-rows (KROW bytes each) -> K^hi, K^lo (exact two-part).
+__device__ __forceinline__ void dequant_k_unit(const uint8_t *rk, int r, int bk, bool in,
+                                               const uint32_t (&off)[4], uint8_t *kh, uint8_t *kl)
+{
+    if (in) {
+        // ---- K block: d (fp16) + 32 int8
+        const uint8_t *src = rk + r * KROW + 34 * bk;
+        uint32_t w[8];
+        uint32_t d16;
+        if ((bk & 1) == 0) {  // block starts 4-byte aligned: d, q0, q1 | ...
+            uint32_t x[9];
+#pragma unroll
+            for (int q = 0; q < 9; ++q)
+                x[q] = lds32(src + 4 * q);
+            d16 = x[0] & 0xFFFFu;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                w[q] = ptx::prmt(x[q], x[q + 1], 0x5432);
+        } else {              // qs start 4-byte aligned
+            d16 = lds16(src);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                w[q] = lds32(src + 2 + 4 * q);
+        }
+        const __half2 d2 = dup_h(d16);
+#pragma unroll
+        for (int m4 = 0; m4 < 4; ++m4) {
+            uint32_t x0[2], x1[2], r0[2], r1[2];
+            k4(w[2 * m4], d2, x0, r0);
+            k4(w[2 * m4 + 1], d2, x1, r1);
+            sts128(kh + off[m4], x0[0], x0[1], x1[0], x1[1]);
+            sts128(kl + off[m4], r0[0], r0[1], r1[0], r1[1]);
+        }
+    } else {
+#pragma unroll
+        for (int m4 = 0; m4 < 4; ++m4) {
+            sts128(kh + off[m4], 0u, 0u, 0u, 0u);
+            sts128(kl + off[m4], 0u, 0u, 0u, 0u);
+        }
+    }
+}
+
+// V: rv = raw Q4_0 head-rows (VROW bytes each) -> V^.
+__device__ __forceinline__ void dequant_v_unit(const uint8_t *rv, int r, int bk, bool in,
+                                               const uint32_t (&off)[4], uint8_t *vh)
+{
+    if (in) {
+        // ---- V block: d (fp16) + 16 bytes of nibbles
+        const uint8_t *vsrc = rv + r * VROW + 18 * bk;
+        uint32_t vw[4];
+        uint32_t d16;
+        if ((bk & 1) == 0) {
+            uint32_t x[5];
+#pragma unroll
+            for (int q = 0; q < 5; ++q)
+                x[q] = lds32(vsrc + 4 * q);
+            d16 = x[0] & 0xFFFFu;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                vw[q] = ptx::prmt(x[q], x[q + 1], 0x5432);
+        } else {
+            d16 = lds16(vsrc);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                vw[q] = lds32(vsrc + 2 + 4 * q);
+        }
+        const __half2 dv = dup_h(d16);
+        // byte j of the block: element j (low nibble), element j + 16 (high)
+        uint32_t lo[8], hi[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            v2(ptx::prmt(vw[q], 0u, 0x4140), dv, lo[2 * q], hi[2 * q]);          // bytes 0, 1
+            v2(ptx::prmt(vw[q], 0u, 0x4342), dv, lo[2 * q + 1], hi[2 * q + 1]);  // bytes 2, 3
+        }
+        sts128(vh + off[0], lo[0], lo[1], lo[2], lo[3]);
+        sts128(vh + off[1], lo[4], lo[5], lo[6], lo[7]);
+        sts128(vh + off[2], hi[0], hi[1], hi[2], hi[3]);
+        sts128(vh + off[3], hi[4], hi[5], hi[6], hi[7]);
+    } else {
+        // keys past the end: zero V so that 0-weight products stay 0
+#pragma unroll
+        for (int m4 = 0; m4 < 4; ++m4)
+            sts128(vh + off[m4], 0u, 0u, 0u, 0u);
+    }
+}
+
+template <bool PRE>
+__global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const PrefillArgs a, int row0)
 {
     extern __shared__ __align__(1024) uint8_t pf_raw[];
     uint8_t *smem = pf_raw + ((1024u - (ptx::smem_u32(pf_raw) & 1023u)) & 1023u);
@@ -177,7 +272,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
             ptx::mbar_init(&hd.raw_free[i], N_DEQ);
         }
         for (int i = 0; i < NB; ++i) {
-            ptx::mbar_init(&hd.k_full[i], N_DEQ);
+            ptx::mbar_init(&hd.k_full[i], PRE ? 1 : N_DEQ);  // PRE: one copy of the whole tile
             ptx::mbar_init(&hd.v_full[i], N_DEQ);
         }
         for (int i = 0; i < NS; ++i) {
@@ -189,6 +284,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         hd.abort = 0;
         ptx::fence_mbar_init();
     }
+    constexpr int W_PROD = w_prod<PRE>(), W_MMA = w_mma<PRE>();
     if (warp == W_MMA) {
         ptx::tmem_alloc(&hd.tmem_base, 512);
         ptx::tmem_relinquish();
@@ -382,42 +478,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
             uint8_t *kh = smem + OFF_KH + kb * TILE_H;
             uint8_t *kl = smem + OFF_KL + kb * TILE_H;
             uint8_t *vh = smem + OFF_VH + kb * TILE_H;
-            if (in) {
-                // ---- K block: d (fp16) + 32 int8
-                const uint8_t *src = rk + r * KROW + 34 * bk;
-                uint32_t w[8];
-                uint32_t d16;
-                if ((bk & 1) == 0) {  // block starts 4-byte aligned: d, q0, q1 | ...
-                    uint32_t x[9];
-#pragma unroll
-                    for (int q = 0; q < 9; ++q)
-                        x[q] = lds32(src + 4 * q);
-                    d16 = x[0] & 0xFFFFu;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        w[q] = ptx::prmt(x[q], x[q + 1], 0x5432);
-                } else {              // qs start 4-byte aligned
-                    d16 = lds16(src);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        w[q] = lds32(src + 2 + 4 * q);
-                }
-                const __half2 d2 = dup_h(d16);
-#pragma unroll
-                for (int m4 = 0; m4 < 4; ++m4) {
-                    uint32_t x0[2], x1[2], r0[2], r1[2];
-                    k4(w[2 * m4], d2, x0, r0);
-                    k4(w[2 * m4 + 1], d2, x1, r1);
-                    sts128(kh + off[m4], x0[0], x0[1], x1[0], x1[1]);
-                    sts128(kl + off[m4], r0[0], r0[1], r1[0], r1[1]);
-                }
-            } else {
-#pragma unroll
-                for (int m4 = 0; m4 < 4; ++m4) {
-                    sts128(kh + off[m4], 0u, 0u, 0u, 0u);
-                    sts128(kl + off[m4], 0u, 0u, 0u, 0u);
-                }
-            }
+            dequant_k_unit(rk, r, bk, in, off, kh, kl);
             ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
             __syncwarp();
             if (lane == 0)
@@ -428,50 +489,45 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
                     fail();
                 break;
             }
-            if (in) {
-                // ---- V block: d (fp16) + 16 bytes of nibbles
-                const uint8_t *vsrc = rv + r * VROW + 18 * bk;
-                uint32_t vw[4];
-                uint32_t d16;
-                if ((bk & 1) == 0) {
-                    uint32_t x[5];
-#pragma unroll
-                    for (int q = 0; q < 5; ++q)
-                        x[q] = lds32(vsrc + 4 * q);
-                    d16 = x[0] & 0xFFFFu;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        vw[q] = ptx::prmt(x[q], x[q + 1], 0x5432);
-                } else {
-                    d16 = lds16(vsrc);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        vw[q] = lds32(vsrc + 2 + 4 * q);
-                }
-                const __half2 dv = dup_h(d16);
-                // byte j of the block: element j (low nibble), element j + 16 (high)
-                uint32_t lo[8], hi[8];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    v2(ptx::prmt(vw[q], 0u, 0x4140), dv, lo[2 * q], hi[2 * q]);          // bytes 0, 1
-                    v2(ptx::prmt(vw[q], 0u, 0x4342), dv, lo[2 * q + 1], hi[2 * q + 1]);  // bytes 2, 3
-                }
-                sts128(vh + off[0], lo[0], lo[1], lo[2], lo[3]);
-                sts128(vh + off[1], lo[4], lo[5], lo[6], lo[7]);
-                sts128(vh + off[2], hi[0], hi[1], hi[2], hi[3]);
-                sts128(vh + off[3], hi[4], hi[5], hi[6], hi[7]);
-            } else {
-                // keys past the end: zero V so that 0-weight products stay 0
-#pragma unroll
-                for (int m4 = 0; m4 < 4; ++m4)
-                    sts128(vh + off[m4], 0u, 0u, 0u, 0u);
-            }
+            dequant_v_unit(rv, r, bk, in, off, vh);
             ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(&hd.raw_free[rb]);
                 ptx::mbar_arrive(&hd.v_full[kb]);
             }
+        }
+    } else if (warp == W_PROD && PRE) {
+        // ================================================================ copies (PRE)
+        // The f16 tiles were expanded into the workspace: tile j of (layer, h) is one
+        // 48 KB image of the three slots.  Slot kb is free once the QK^T (K^) and the
+        // PV (V^) of tile j - NB are done; one transaction barrier covers the tile.
+        if (lane == 0) {
+            const int tiles_total = (int)((a.n_cached + a.T + BN - 1) / BN);
+            const uint8_t *wsb = static_cast<const uint8_t *>(a.workspace) +
+                                 ((int64_t)layer * a.n_kv_heads + h) * tiles_total * TILE3;
+            int issued = 0;
+            for (int j = 0; j < ntiles; ++j) {
+                const int kb = slot(j, NB);
+                if (*abort || (j >= NB && (!ptx::mbar_wait_bounded(&hd.s_full[slot(j - NB, NS)],
+                                                                   par(j - NB, NS), abort, WAIT_NS) ||
+                                           !ptx::mbar_wait_bounded(&hd.pv_done[slot(j - NB, NS)],
+                                                                   par(j - NB, NS), abort, WAIT_NS)))) {
+                    fail();
+                    break;
+                }
+                const uint8_t *src = wsb + (int64_t)j * TILE3;
+                ptx::mbar_arrive_expect_tx(&hd.k_full[kb], TILE3);
+                ptx::bulk_g2s(smem + OFF_KH + kb * TILE_H, src, TILE_H, &hd.k_full[kb]);
+                ptx::bulk_g2s(smem + OFF_KL + kb * TILE_H, src + TILE_H, TILE_H, &hd.k_full[kb]);
+                ptx::bulk_g2s(smem + OFF_VH + kb * TILE_H, src + 2 * TILE_H, TILE_H, &hd.k_full[kb]);
+                issued = j + 1;
+            }
+            // no copy may still be landing when the CTA exits
+            int none = 0;
+            for (int j = (issued > NB ? issued - NB : 0); j < issued; ++j)
+                if (!ptx::mbar_wait_bounded(&hd.k_full[slot(j, NB)], par(j, NB), &none, WAIT_NS))
+                    report_timeout(a.status);
         }
     } else if (warp == W_PROD) {
         // ================================================================ copies
@@ -518,7 +574,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
         // and waits for v_full itself
         auto issue_pv = [&](int jj) -> bool {
             const int vb = slot(jj, NB), sb = slot(jj, NS);
-            if ((jj == ntiles - 1 && !wwait(&hd.v_full[vb], par(jj, NB))) ||
+            if ((!PRE && jj == ntiles - 1 && !wwait(&hd.v_full[vb], par(jj, NB))) ||
                 !wwait(&hd.p_full[sb], par(jj, NS)))
                 return false;
             ptx::tc_fence_after();
@@ -578,6 +634,65 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_tc_kernel(const Prefill
     if (warp == W_MMA) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tbase, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Expansion of the f16 tiles into the workspace, once per call: one CTA per
+// (key tile, KV head, layer) copies the tile's raw rows in, dequantizes them with
+// the same unit routines as the dequant warps (so the tiles are bit-identical),
+// and stores the 48 KB image of the three slots (K^hi, K^lo, V^, 128-byte
+// swizzle) with one bulk copy.  The prefill kernel then bulk-copies each tile
+// straight into its slots: every row tile of a KV head reads the same keys, and
+// this turns 96 dequantizations of a key tile (prefill262k) into one.
+constexpr int EXP_THREADS = N_DEQ * 32;  // one K unit and one V unit per thread
+constexpr int EXP_SMEM = TILE3 + RAW_BYTES + 16 + 1024;
+
+__global__ void __launch_bounds__(EXP_THREADS) prefill_expand_kernel(const PrefillArgs a,
+                                                                     int tiles_total)
+{
+    extern __shared__ __align__(1024) uint8_t ex_raw_sm[];
+    uint8_t *smem = ex_raw_sm + ((1024u - (ptx::smem_u32(ex_raw_sm) & 1023u)) & 1023u);
+    uint8_t *kh = smem, *kl = smem + TILE_H, *vh = smem + 2 * TILE_H;
+    uint8_t *rk = smem + TILE3, *rv = rk + RAW_K;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + TILE3 + RAW_BYTES);
+    __shared__ int ok_s;
+    const int t = blockIdx.x, h = blockIdx.y, layer = blockIdx.z;
+    const int64_t n_keys = a.n_cached + a.T;
+    const int rows = (int)min((int64_t)BN, n_keys - (int64_t)t * BN);
+    const int64_t cap = a.layers.cap[layer];
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+        ptx::mbar_arrive_expect_tx(bar, rows * (KROW + VROW));
+        ptx::bulk_g2s(rk, a.layers.k[layer] + ((int64_t)h * cap + (int64_t)t * BN) * KROW,
+                      rows * KROW, bar);
+        ptx::bulk_g2s(rv, a.layers.v[layer] + ((int64_t)h * cap + (int64_t)t * BN) * VROW,
+                      rows * VROW, bar);
+        int none = 0;
+        ok_s = ptx::mbar_wait_bounded(bar, 0, &none, WAIT_NS) ? 1 : 0;
+        if (!ok_s)
+            report_timeout(a.status);
+    }
+    __syncthreads();
+    if (!ok_s)
+        return;  // the copy timed out (recorded); it was waited for as long as allowed
+    const int grp = threadIdx.x >> 5, ln = threadIdx.x & 31;
+    const int r = (grp % (BN / 8)) * 8 + (ln & 7), bk = grp / (BN / 8) + 2 * (ln >> 3);
+    uint32_t off[4];
+#pragma unroll
+    for (int m4 = 0; m4 < 4; ++m4)
+        off[m4] = sw_off(r, 32 * bk + 8 * m4);
+    dequant_k_unit(rk, r, bk, r < rows, off, kh, kl);
+    dequant_v_unit(rv, r, bk, r < rows, off, vh);
+    ptx::fence_proxy_async_smem();  // generic-proxy writes -> the bulk store reads them
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint8_t *dst = static_cast<uint8_t *>(a.workspace) +
+                       (((int64_t)layer * a.n_kv_heads + h) * tiles_total + t) * TILE3;
+        ptx::bulk_s2g(dst, smem, TILE3);
+        ptx::bulk_commit();
+        ptx::bulk_wait_read0();  // the shared memory stays valid until it has been read
     }
 }
 
@@ -696,6 +811,13 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
 
 size_t prefill_workspace_bytes(int, int, int, int, int) { return 0; }
 
+size_t prefill_expand_bytes(int n_layers, int n_kv_heads, int head_dim, int64_t n_keys)
+{
+    if (head_dim != HD || n_layers < 1 || n_kv_heads < 1 || n_keys < 1)
+        return 0;
+    return (size_t)n_layers * n_kv_heads * (size_t)((n_keys + BN - 1) / BN) * TILE3;
+}
+
 bool prefill_supported(int n_q_heads, int n_kv_heads, int head_dim)
 {
     const int G = n_q_heads / n_kv_heads;
@@ -730,18 +852,34 @@ void launch_prefill(const PrefillArgs &a, cudaStream_t s)
         prefill_exact_kernel<<<grid, EX_THREADS, smem, s>>>(a, tb, (int)t_split);
     }
     if (t_split < a.T) {
-        static bool attr_tc[64] = {};
+        // with a workspace (the caller checked its size), expand the f16 tiles once
+        const bool pre = a.workspace != nullptr;
+        static bool attr_tc[2][64] = {};
         int dev = 0;
         cudaGetDevice(&dev);
-        if (dev >= 0 && dev < 64 && !attr_tc[dev]) {
-            cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 PF_SMEM);
-            attr_tc[dev] = true;
+        if (dev >= 0 && dev < 64 && !attr_tc[pre][dev]) {
+            if (pre) {
+                cudaFuncSetAttribute(prefill_tc_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM);
+                cudaFuncSetAttribute(prefill_expand_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, EXP_SMEM);
+            } else {
+                cudaFuncSetAttribute(prefill_tc_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM);
+            }
+            attr_tc[pre][dev] = true;
         }
         const int row0 = (int)t_split * G;
         const int rows = a.T * G - row0;
         dim3 grid((unsigned)((rows + BM - 1) / BM), a.n_kv_heads, a.n_layers);
-        prefill_tc_kernel<<<grid, PF_THREADS, PF_SMEM, s>>>(a, row0);
+        if (pre) {
+            const int tiles_total = (int)((a.n_cached + a.T + BN - 1) / BN);
+            dim3 egrid((unsigned)tiles_total, a.n_kv_heads, a.n_layers);
+            prefill_expand_kernel<<<egrid, EXP_THREADS, EXP_SMEM, s>>>(a, tiles_total);
+            prefill_tc_kernel<true><<<grid, pf_threads<true>(), PF_SMEM, s>>>(a, row0);
+        } else {
+            prefill_tc_kernel<false><<<grid, pf_threads<false>(), PF_SMEM, s>>>(a, row0);
+        }
     }
 }
 

@@ -109,6 +109,24 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// ---- bulk async copy shared -> global (bulk-group completion) -----------------
+// src 16-byte aligned shared memory, dst 16-byte aligned global, bytes a multiple
+// of 16.  Writers of src must have issued fence_proxy_async_smem() (and synced)
+// first; bulk_wait_read0() returns once every committed store has read its source.
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+__device__ __forceinline__ void bulk_wait_read0()
+{
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // ---- named barriers ---------------------------------------------------------
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads)

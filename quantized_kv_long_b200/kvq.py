@@ -82,6 +82,7 @@ _SIGS = {
     "kvq_decode_merged_static": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P],
                                  _I32),
     "kvq_resident_layers": ([_SZ, _I32, _I64, _I32, _I32, _I32, _I32], _I32),
+    "kvq_prefill_workspace_bytes": ([_I32, _I32, _I32, _I64], _SZ),
     "kvq_workspace_bytes": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "kvq_check": ([_P], _I32),
     "kvq_status_string": ([_I32], ctypes.c_char_p),
@@ -184,6 +185,8 @@ def kvq_prefill_attn(layers, q, n_q_heads: int, T: int, n_cached: int, page: int
                      out, lse, page_out=None, page_lse=None, workspace=None, ws_bytes: int = 0,
                      stream=None) -> None:
     arr, n = _layers(layers)
+    if workspace is not None and not ws_bytes and isinstance(workspace, torch.Tensor):
+        ws_bytes = workspace.numel() * workspace.element_size()
     _check(_lib.kvq_prefill_attn(arr, n, _ptr(q), n_q_heads, T, n_cached, page, scale,
                                  _ptr(out), _ptr(lse), _ptr(page_out), _ptr(page_lse),
                                  _ptr(workspace), ws_bytes, _stream(stream)))
@@ -217,6 +220,11 @@ def kvq_resident_layers(budget_bytes: int, n_layers: int, capacity: int, n_kv_he
                         head_dim: int, k_type: int = 0, v_type: int = 0) -> int:
     return _lib.kvq_resident_layers(budget_bytes, n_layers, capacity, n_kv_heads, head_dim,
                                     k_type, v_type)
+
+
+def kvq_prefill_workspace_bytes(n_layers: int, n_kv_heads: int, head_dim: int,
+                                n_keys: int) -> int:
+    return _lib.kvq_prefill_workspace_bytes(n_layers, n_kv_heads, head_dim, n_keys)
 
 
 def kvq_workspace_bytes(op: int, n_layers: int, n_q_heads: int, n_kv_heads: int, T: int,

@@ -210,3 +210,18 @@ def test_block_format_validation(kvq):
     assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 1, 1) == 3
     assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 0, 0) == 4
     assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 7, 0) == -1
+
+
+def test_prefill_workspace_validation(kvq):
+    """The optional prefill workspace: its size for the expanded f16 key tiles, and a
+    too-small or misaligned one refused before anything is launched."""
+    nb = kvq.kvq_prefill_workspace_bytes(16, 4, 256, 264192)
+    assert nb == 16 * 4 * 8256 * 49152
+    assert kvq.kvq_prefill_workspace_bytes(1, 4, 128, 1000) == 0  # no tensor-core path
+    L = _layer(kvq, capacity=4096)
+    need = kvq.kvq_prefill_workspace_bytes(1, 4, 256, 1024 + 128)
+    args = (L, A, 24, 128, 1024, 1024, 1 / 16, A, A)
+    _raises(kvq, kvq.KVQ_ERR_WORKSPACE, kvq.kvq_prefill_attn, *args, workspace=A,
+            ws_bytes=need - 1)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_prefill_attn, *args, workspace=A + 16,
+            ws_bytes=need)

@@ -23,12 +23,17 @@ def kvq():
     return m
 
 
-def run_prefill(kvq, cache, q, Hq, T, n_cached, scale, page=1024):
+def run_prefill(kvq, cache, q, Hq, T, n_cached, scale, page=1024, expand=False):
+    """expand: pass a workspace, so that the key tiles are expanded once per call."""
     L, D = q.shape[0], q.shape[-1]
     out = torch.full((L, T, Hq, D), float("nan"), device="cuda")
     lse = torch.full((L, T, Hq), float("nan"), device="cuda")
+    ws = None
+    if expand:
+        nb = kvq.kvq_prefill_workspace_bytes(L, cache.n_kv_heads, D, n_cached + T)
+        ws = torch.full((max(nb, 1),), 0x7F, dtype=torch.uint8, device="cuda")  # garbage
     kvq.kvq_prefill_attn(cache.layers(), torch.from_numpy(q).cuda(), Hq, T, n_cached, page, scale,
-                         out, lse)
+                         out, lse, workspace=ws)
     kvq.kvq_check()
     return out.cpu().numpy(), lse.cpu().numpy()
 
@@ -43,6 +48,9 @@ def check(kvq, w, n_layers, T, n_cached):
     for l in layers:
         ro, rl = oracle.prefill_attn(orc[l][0], orc[l][1], q[l], n_cached, 1024, w.scale)
         assert_attn_close(out[l], lse[l], ro, rl, f"prefill layer {l}")
+    # the expanded-tile path (workspace) gives the same bits
+    eo, el = run_prefill(kvq, cache, q, w.n_q_heads, T, n_cached, w.scale, expand=True)
+    assert np.array_equal(eo, out) and np.array_equal(el, lse), "workspace path differs"
 
 
 def test_tensor_core_path(kvq):
@@ -81,10 +89,19 @@ def test_prefill262k_full_size_sampled(kvq):
     q = np.stack([wl.q_rows(w, l) for l in range(w.n_layers)])
     out = torch.full((w.n_layers, T, Hq, 256), float("nan"), device=device)
     lse = torch.full((w.n_layers, T, Hq), float("nan"), device=device)
-    kvq.kvq_prefill_attn(cache.layers(), torch.from_numpy(q).cuda(), Hq, T, nc, w.page, w.scale,
-                         out, lse)
+    qd = torch.from_numpy(q).cuda()
+    kvq.kvq_prefill_attn(cache.layers(), qd, Hq, T, nc, w.page, w.scale, out, lse)
     kvq.kvq_check()
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    # the launch the benchmark times: with the expanded-tile workspace (26 GB), same bits
+    nb = kvq.kvq_prefill_workspace_bytes(w.n_layers, w.n_kv_heads, 256, nc + T)
+    ws = torch.empty((nb,), dtype=torch.uint8, device=device)
+    out2 = torch.full_like(out, float("nan"))
+    lse2 = torch.full_like(lse, float("nan"))
+    kvq.kvq_prefill_attn(cache.layers(), qd, Hq, T, nc, w.page, w.scale, out2, lse2, workspace=ws)
+    kvq.kvq_check()
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+    del ws, out2, lse2
     rng = np.random.default_rng(7)
     for l in (0, 9):
         kc, vc = oracle.empty_cache(w.n_kv_heads, w.head_dim, nc + T)
