@@ -66,13 +66,19 @@ constexpr int KROW = 272, VROW = 144;
 constexpr int RAW_K = BN * KROW, RAW_V = BN * VROW, RAW_BYTES = RAW_K + RAW_V;  // 13,312 B
 constexpr int TILE_H = BN * HD * 2;  // one f16 tile of 32 keys x 256 dims: 16 KB
 constexpr int NR = 4;  // raw staging slots (bulk copies in flight ahead of the dequant)
-constexpr int NB = 3;  // f16 K^hi / K^lo / V^ tile slots
+// f16 K^hi / K^lo / V^ tile slots: 3 beside the raw staging ring, 4 when the tiles
+// come expanded from the workspace (no raw ring, and one more tile of copy lead)
+template <bool PRE> constexpr int nb() { return PRE ? 4 : 3; }
+constexpr int NB_MAX = 4;
 constexpr int NS = 4;  // S / P slots in tensor memory
 constexpr int N_SOFT = 4, N_DEQ = 8;
 // roles: softmax warps, dequant warps (none when the f16 tiles were expanded into
 // the workspace beforehand), the producer warp, the MMA warp
 template <bool PRE> constexpr int n_deq() { return PRE ? 0 : N_DEQ; }
-template <bool PRE> constexpr int w_prod() { return N_SOFT + n_deq<PRE>(); }
+// softmax warps: one per TMEM lane quadrant, or two (each with half of a tile's keys)
+// when no dequant warps compete for the issue slots
+template <bool PRE> constexpr int n_soft() { return PRE ? 2 * N_SOFT : N_SOFT; }
+template <bool PRE> constexpr int w_prod() { return n_soft<PRE>() + n_deq<PRE>(); }
 template <bool PRE> constexpr int w_mma() { return w_prod<PRE>() + 1; }
 template <bool PRE> constexpr int pf_threads() { return (w_mma<PRE>() + 1) * 32; }  // 14 / 6 warps
 constexpr int TILE3 = 3 * TILE_H;  // one key tile's K^hi, K^lo, V^ in the workspace: 48 KB
@@ -86,25 +92,36 @@ constexpr float M_INIT = -1.0e30f;
 constexpr uint32_t COL_O = 0, COL_Q = 256, COL_S0 = 384;
 static_assert(COL_S0 + NS * BN <= 512, "tensor-memory columns");
 static_assert(BN * 8 == N_DEQ * 32, "one K unit and one V unit per dequant thread and tile");
-static_assert(NB <= NS, "a K^ slot is reused only after the QK^T that read it");
-// The MMA warp waits only for k_full(j) and p_full(j - 1) per tile.  k_full(j)
-// completes after every dequant warp has finished V^ of tile j - 1 (program order
-// in each warp), which in turn waited for the PV of tile j - 1 - NB = j - NS to
-// finish; so k_full(j) also covers v_full(j - 1) and the S/P slot of tile j.
-static_assert(NS == NB + 1, "k_full(j) must imply that the PV of tile j - NS is done");
+// The MMA warp waits only for k_full(j) and p_full(j - 1) per tile, and k_full(j)
+// must imply that the PV of tile j - NS (which read the S/P slot the QK^T of tile j
+// rewrites) is done.  PVs finish in order.
+//  - Dequant warps: k_full(j) completes after every dequant warp has finished V^ of
+//    tile j - 1 (program order in each warp), which waited for the PV of tile
+//    j - 1 - NB; so k_full(j) covers v_full(j - 1) too.  Needs NB + 1 <= NS.
+//  - Expanded tiles: the producer copies tile j after the PV of tile j - NB is done.
+//    Needs NB <= NS.
+static_assert(nb<false>() + 1 <= NS && nb<true>() <= NS, "k_full(j): the PV of tile j - NS");
 
 struct PfSmemHead {
-    uint64_t raw_full[NR], raw_free[NR], k_full[NB], v_full[NB], s_full[NS], p_full[NS],
+    uint64_t raw_full[NR], raw_free[NR], k_full[NB_MAX], v_full[NB_MAX], s_full[NS], p_full[NS],
         pv_done[NS], q_ready;
+    uint64_t xch[N_SOFT];            // two softmax warps per quadrant: per-tile exchange
+    float xmx[2][2][BM];             // [warp half][phase parity][row]: tile max, then l
     uint32_t tmem_base;
     int abort;
 };
-// layout: [K^hi NB x 16K][K^lo NB x 16K][V^ NB x 16K][raw NR x 13,312][head], base 1024-aligned
-constexpr int OFF_KH = 0, OFF_KL = NB * TILE_H, OFF_VH = 2 * NB * TILE_H;
-constexpr int OFF_RAW = 3 * NB * TILE_H;
-constexpr int OFF_HEAD = OFF_RAW + NR * RAW_BYTES;
-constexpr int PF_SMEM = OFF_HEAD + (int)sizeof(PfSmemHead) + 1024;  // + alignment slack
-static_assert(PF_SMEM <= 232448, "dynamic shared memory per block");
+// layout: [K^hi NB x 16K][K^lo NB x 16K][V^ NB x 16K][raw NR x 13,312 (dequant warps
+// only)][head], base 1024-aligned
+template <bool PRE> constexpr int off_head()
+{
+    return 3 * nb<PRE>() * TILE_H + (PRE ? 0 : NR * RAW_BYTES);
+}
+template <bool PRE> constexpr int pf_smem()
+{
+    return off_head<PRE>() + (int)sizeof(PfSmemHead) + 1024;  // + alignment slack
+}
+static_assert(pf_smem<false>() <= 232448 && pf_smem<true>() <= 232448,
+              "dynamic shared memory per block");
 
 // slot and phase parity of tile t in a ring of S slots
 __device__ __forceinline__ int slot(int t, int S) { return t % S; }
@@ -252,6 +269,9 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
 {
     extern __shared__ __align__(1024) uint8_t pf_raw[];
     uint8_t *smem = pf_raw + ((1024u - (ptx::smem_u32(pf_raw) & 1023u)) & 1023u);
+    constexpr int NB = nb<PRE>();
+    constexpr int OFF_KH = 0, OFF_KL = NB * TILE_H, OFF_VH = 2 * NB * TILE_H;
+    constexpr int OFF_RAW = 3 * NB * TILE_H, OFF_HEAD = off_head<PRE>();
     PfSmemHead &hd = *reinterpret_cast<PfSmemHead *>(smem + OFF_HEAD);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.n_q_heads / a.n_kv_heads;
@@ -277,10 +297,12 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         }
         for (int i = 0; i < NS; ++i) {
             ptx::mbar_init(&hd.s_full[i], 1);
-            ptx::mbar_init(&hd.p_full[i], N_SOFT);
+            ptx::mbar_init(&hd.p_full[i], n_soft<PRE>());
             ptx::mbar_init(&hd.pv_done[i], 1);
         }
-        ptx::mbar_init(&hd.q_ready, N_SOFT);
+        ptx::mbar_init(&hd.q_ready, n_soft<PRE>());
+        for (int i = 0; i < N_SOFT; ++i)
+            ptx::mbar_init(&hd.xch[i], 2);
         hd.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -307,19 +329,36 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     };
 
-    if (warp < N_SOFT) {
+    if (warp < n_soft<PRE>()) {
         // ================================================================ softmax
-        const int i = warp * 32 + lane;  // query row of this thread = its TMEM lane
+        // Warp (quad, hf) owns the query rows of TMEM lane quadrant quad (one row per
+        // thread).  With NH = 2 warps per quadrant, warp hf takes keys [16 hf, 16 hf + 16)
+        // of every tile and columns [128 hf, 128 hf + 128) of O; the pair agrees on the
+        // running max through hd.xch / hd.xmx once per tile.  The arithmetic does not
+        // depend on NH: each 16-key half of a tile has its own running sum l[hh],
+        // l = l[0] + l[1] at the end, and the max is exact.
+        constexpr int NH = n_soft<PRE>() / N_SOFT;
+        const int quad = warp & 3, hf = warp >> 2;
+        const int h0 = NH == 2 ? hf : 0;  // this warp's halves: [h0, h0 + 2 / NH)
+        const int i = quad * 32 + lane;   // query row of this thread = its TMEM lane
         const int gr = R0 + i;
         const bool live = gr <= r_last;
         const int t = live ? gr / G : 0, gq = live ? gr % G : 0;
         const int64_t lim = a.n_cached + t;  // last visible key
-        const uint32_t lane_addr = tbase + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_addr = tbase + ((uint32_t)(quad * 32) << 16);
+        // bounded wait on the pair's exchange barrier (phase ph); false: give up
+        auto pair_sync = [&](uint32_t ph) -> bool {
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                ptx::mbar_arrive(&hd.xch[quad]);
+            return wwait(&hd.xch[quad], ph & 1u);
+        };
         {   // Q row -> TMEM columns [COL_Q, COL_Q + 128): two f16 per column, lower dim low
             const uint4 *qp = reinterpret_cast<const uint4 *>(
                 a.q + (((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq) * HD);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = h0 * 4; c < h0 * 4 + 8 / NH; ++c) {
                 uint32_t r[16];
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
@@ -338,59 +377,71 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                 ptx::mbar_arrive(&hd.q_ready);
         }
         const float sl2 = a.scale * LOG2E;
-        float m = M_INIT, l = 0.0f;
-        for (int j = 0; j < ntiles; ++j) {
+        constexpr int NHALF = 2 / NH;       // 16-key halves whose P and l this warp makes
+        float m = M_INIT, l[NHALF];         // l[k]: running sum of half h0 + k
+#pragma unroll
+        for (int k = 0; k < NHALF; ++k)
+            l[k] = 0.0f;
+        bool ok = true;
+        for (int j = 0; ok && j < ntiles; ++j) {
             const int sb = slot(j, NS);
             const uint32_t scol = COL_S0 + BN * sb;
             if (!wwait(&hd.s_full[sb], par(j, NS))) {
-                if (lane == 0)
-                    fail();
+                ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            float s[BN];
+            // every warp reads the whole tile's scores, so that both warps of a quadrant
+            // take the same max without talking to each other; s[0] holds this warp's
+            // first half (h0), s[1] the other one
+            float s[2][16];
 #pragma unroll
-            for (int c = 0; c < BN / 16; ++c) {
+            for (int k = 0; k < 2; ++k) {
                 uint32_t r[16];
-                ptx::tmem_ld16(lane_addr + scol + 16 * c, r);
-                ptx::tmem_wait_ld();
+                ptx::tmem_ld16(lane_addr + scol + 16 * (k == 0 ? h0 : 1 - h0), r);
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    s[16 * c + e] = __uint_as_float(r[e]) * sl2;
+                    s[k][e] = __uint_as_float(r[e]);
             }
+            ptx::tmem_wait_ld();
             const int64_t kj0 = (int64_t)j * BN;
             if (kj0 + BN - 1 > lim) {  // causal edge / end of the keys
 #pragma unroll
-                for (int e = 0; e < BN; ++e)
-                    if (kj0 + e > lim)
-                        s[e] = -INFINITY;
+                for (int k = 0; k < 2; ++k) {
+                    const int64_t kb0 = kj0 + 16 * (k == 0 ? h0 : 1 - h0);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (kb0 + e > lim)
+                            s[k][e] = -INFINITY;
+                }
             }
-            // tree reduction (independent chains) for the tile max
             float mx8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                mx8[e] = s[e];
+                mx8[e] = fmaxf(s[0][e], s[0][e + 8]);
 #pragma unroll
-            for (int e = 8; e < BN; ++e)
-                mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            for (int e = 0; e < 16; ++e)
+                mx8[e & 7] = fmaxf(mx8[e & 7], s[1][e]);
+            // scaling is monotonic: the max of the scaled scores
+            const float mx = sl2 * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             float alpha = 1.0f;
-            if (mx > m + TAU) {
+            if (mx > m + TAU) {  // lazy running max: moves only by more than TAU
                 alpha = ptx::ex2(m - mx);
                 m = mx;
-                l *= alpha;
+#pragma unroll
+                for (int k = 0; k < NHALF; ++k)
+                    l[k] *= alpha;
             }
-            // rescale O (rare): the whole warp takes part once any lane needs it, after
-            // the PV of the previous tile has finished
+            // rescale this warp's columns of O (rare): the whole warp takes part once any
+            // lane needs it, after the PV of the previous tile has finished
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
                 if (!wwait(&hd.pv_done[slot(j - 1, NS)], par(j - 1, NS))) {
-                    if (lane == 0)
-                        fail();
+                    ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                for (int c = 0; c < 16; ++c) {
+                for (int c = h0 * 8; c < h0 * 8 + 16 / NH; ++c) {
                     uint32_t r[16];
                     ptx::tmem_ld16(lane_addr + COL_O + 16 * c, r);
                     ptx::tmem_wait_ld();
@@ -401,34 +452,48 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                 }
                 ptx::tmem_wait_st();
             }
-            // P = 2^(s - m) in f16 (keys 2e, 2e + 1 in column e) over the first BN / 2
-            // columns of this S slot
-            uint32_t pk[BN / 2];
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            // P = 2^(s scale - m) in f16 (keys 2e, 2e + 1 of half hh in column 8 hh + e of
+            // this S slot), and the half's sum
 #pragma unroll
-            for (int e = 0; e < BN / 2; ++e) {
-                const float p0 = ptx::ex2(s[2 * e] - m), p1 = ptx::ex2(s[2 * e + 1] - m);
-                ls[e & 3] += p0 + p1;
-                pk[e] = ptx::h2_bits(__floats2half2_rn(p0, p1));
+            for (int k = 0; k < NHALF; ++k) {
+                const float *sh = s[k];  // half h0 + k
+                uint32_t pk[8];
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float p0 = ptx::ex2(fmaf(sh[2 * e], sl2, -m));
+                    const float p1 = ptx::ex2(fmaf(sh[2 * e + 1], sl2, -m));
+                    ls[e & 3] += p0 + p1;
+                    pk[e] = ptx::h2_bits(__floats2half2_rn(p0, p1));
+                }
+                l[k] += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                ptx::tmem_st8(lane_addr + scol + 8 * (h0 + k), pk);
             }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            static_assert(BN / 2 == 16, "P of one tile is one 16-column TMEM store");
-            ptx::tmem_st16(lane_addr + scol, pk);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 ptx::mbar_arrive(&hd.p_full[sb]);
         }
-        // ---- epilogue: out = O / l, lse = (m + log2 l) ln 2
-        if (!*abort) {
+        if (!ok && lane == 0)
+            fail();
+        // ---- epilogue: out = O / l, lse = (m + log2 l) ln 2, l = l[0] + l[1]
+        if (ok && !*abort) {
             const int last = ntiles - 1;
-            if (wwait(&hd.pv_done[slot(last, NS)], par(last, NS))) {
+            bool done = wwait(&hd.pv_done[slot(last, NS)], par(last, NS));
+            float lt = l[0] + l[NHALF - 1];  // NH == 1: l of half 0 + l of half 1
+            if (NH == 2 && done) {  // the pair adds its two halves, half 0 first
+                hd.xmx[hf][0][i] = l[0];
+                done = pair_sync(0);
+                if (done)
+                    lt = hd.xmx[0][0][i] + hd.xmx[1][0][i];
+            }
+            if (done) {
                 ptx::tc_fence_after();
-                const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+                const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
                 float4 *op = reinterpret_cast<float4 *>(
                     a.out + (((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq) * HD);
-                for (int c = 0; c < 16; ++c) {
+                for (int c = h0 * 8; c < h0 * 8 + 16 / NH; ++c) {
                     uint32_t r[16];
                     ptx::tmem_ld16(lane_addr + COL_O + 16 * c, r);
                     ptx::tmem_wait_ld();
@@ -441,9 +506,9 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                                                         __uint_as_float(r[4 * v + 3]) * inv);
                     }
                 }
-                if (live)
+                if (live && h0 == 0)
                     a.lse[((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq] =
-                        l > 0.0f ? (m + log2f(l)) * LN2 : -INFINITY;
+                        lt > 0.0f ? (m + log2f(lt)) * LN2 : -INFINITY;
             } else if (lane == 0) {
                 fail();
             }
@@ -860,12 +925,12 @@ void launch_prefill(const PrefillArgs &a, cudaStream_t s)
         if (dev >= 0 && dev < 64 && !attr_tc[pre][dev]) {
             if (pre) {
                 cudaFuncSetAttribute(prefill_tc_kernel<true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM);
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, pf_smem<true>());
                 cudaFuncSetAttribute(prefill_expand_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, EXP_SMEM);
             } else {
                 cudaFuncSetAttribute(prefill_tc_kernel<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM);
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, pf_smem<false>());
             }
             attr_tc[pre][dev] = true;
         }
@@ -876,9 +941,9 @@ void launch_prefill(const PrefillArgs &a, cudaStream_t s)
             const int tiles_total = (int)((a.n_cached + a.T + BN - 1) / BN);
             dim3 egrid((unsigned)tiles_total, a.n_kv_heads, a.n_layers);
             prefill_expand_kernel<<<egrid, EXP_THREADS, EXP_SMEM, s>>>(a, tiles_total);
-            prefill_tc_kernel<true><<<grid, pf_threads<true>(), PF_SMEM, s>>>(a, row0);
+            prefill_tc_kernel<true><<<grid, pf_threads<true>(), pf_smem<true>(), s>>>(a, row0);
         } else {
-            prefill_tc_kernel<false><<<grid, pf_threads<false>(), PF_SMEM, s>>>(a, row0);
+            prefill_tc_kernel<false><<<grid, pf_threads<false>(), pf_smem<false>(), s>>>(a, row0);
         }
     }
 }

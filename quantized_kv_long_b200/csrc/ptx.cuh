@@ -286,6 +286,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7])
+        : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (atoms of 8 rows x 128 B,
 // 1024-byte aligned).  lbo / sbo in bytes.
 __device__ __forceinline__ uint64_t smem_desc_sw128(const void *p, uint32_t lbo, uint32_t sbo)
