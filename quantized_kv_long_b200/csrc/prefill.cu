@@ -105,7 +105,8 @@ static_assert(nb<false>() + 1 <= NS && nb<true>() <= NS, "k_full(j): the PV of t
 struct PfSmemHead {
     uint64_t raw_full[NR], raw_free[NR], k_full[NB_MAX], v_full[NB_MAX], s_full[NS], p_full[NS],
         pv_done[NS], q_ready;
-    uint64_t xch[N_SOFT];            // two softmax warps per quadrant: per-tile exchange
+    uint64_t mma_drain;              // one commit after the last MMA: all of them are done
+    uint64_t xch[N_SOFT];            // two softmax warps per quadrant: the final sums
     float xmx[2][2][BM];             // [warp half][phase parity][row]: tile max, then l
     uint32_t tmem_base;
     int abort;
@@ -301,6 +302,7 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
             ptx::mbar_init(&hd.pv_done[i], 1);
         }
         ptx::mbar_init(&hd.q_ready, n_soft<PRE>());
+        ptx::mbar_init(&hd.mma_drain, 1);
         for (int i = 0; i < N_SOFT; ++i)
             ptx::mbar_init(&hd.xch[i], 2);
         hd.abort = 0;
@@ -625,6 +627,19 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         // elected lane issues every MMA and commit, so all tcgen05 work of the
         // CTA comes from one thread and each commit covers what came before.
         const uint32_t leader = ptx::elect_one();
+        // the MMA warp's waits: every lane tests the barrier without blocking (no
+        // lane-divergent branch, no broadcast), bounded in time and by the abort flag
+        auto mwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            if (ptx::mbar_test(bar, parity))
+                return true;
+            const uint64_t t0 = ptx::globaltimer_ns();
+            for (;;) {
+                if (ptx::mbar_test(bar, parity))
+                    return true;
+                if (*abort || ptx::globaltimer_ns() - t0 > WAIT_NS)
+                    return false;
+            }
+        };
         const uint32_t id_qk = ptx::idesc_f16_f32(BM, BN, false, false);
         const uint32_t id_pv = ptx::idesc_f16_f32(BM, HD, false, true);
         // descriptors of slot 0; slots and k-steps add to the start-address field
@@ -632,15 +647,14 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         const uint64_t dk_hi0 = ptx::smem_desc_sw128(smem + OFF_KH, 16, 1024);
         const uint64_t dk_lo0 = ptx::smem_desc_sw128(smem + OFF_KL, 16, 1024);
         const uint64_t dv0 = ptx::smem_desc_sw128(smem + OFF_VH, BN * 128, 1024);
-        int committed = -1;  // last tile whose PV was committed
         bool ok = wwait(&hd.q_ready, 0);
         // PV of tile jj, issued after the QK^T of tile jj + 1: V^ is ready once
         // k_full(jj + 1) has completed (see NS above); the last tile has no successor
         // and waits for v_full itself
         auto issue_pv = [&](int jj) -> bool {
             const int vb = slot(jj, NB), sb = slot(jj, NS);
-            if ((!PRE && jj == ntiles - 1 && !wwait(&hd.v_full[vb], par(jj, NB))) ||
-                !wwait(&hd.p_full[sb], par(jj, NS)))
+            if ((!PRE && jj == ntiles - 1 && !mwait(&hd.v_full[vb], par(jj, NB))) ||
+                !mwait(&hd.p_full[sb], par(jj, NS)))
                 return false;
             ptx::tc_fence_after();
             if (leader) {
@@ -652,14 +666,13 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                 ptx::umma_commit(&hd.pv_done[sb]);
             }
             __syncwarp();
-            committed = jj;
             return true;
         };
         for (int j = 0; ok && j < ntiles; ++j) {
             const int kb = slot(j, NB), sb = slot(j, NS);
             // K^ of tile j is ready, and (see NS above) the PV of tile j - NS that read
             // S/P slot sb is done
-            ok = wwait(&hd.k_full[kb], par(j, NB));
+            ok = mwait(&hd.k_full[kb], par(j, NB));
             if (!ok)
                 break;
             ptx::tc_fence_after();
@@ -684,12 +697,14 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
             ok = issue_pv(ntiles - 1);
         if (!ok && lane == 0)
             fail();
-        // every committed MMA has finished before TMEM is freed (a commit tracks all
-        // earlier tcgen05 operations of the issuing thread)
+        // every issued MMA has finished before TMEM is freed, also after a failed wait:
+        // one commit tracks all earlier tcgen05 operations of the issuing thread
+        if (leader)
+            ptx::umma_commit(&hd.mma_drain);
+        __syncwarp();
         if (lane == 0) {
             int none = 0;
-            if (committed >= 0 && !ptx::mbar_wait_bounded(&hd.pv_done[slot(committed, NS)],
-                                                          par(committed, NS), &none, WAIT_NS))
+            if (!ptx::mbar_wait_bounded(&hd.mma_drain, 0, &none, WAIT_NS))
                 report_timeout(a.status);
         }
         __syncwarp();
