@@ -340,7 +340,8 @@ def run_ours(args, w: wl.Workload) -> dict | None:
     return res
 
 
-DECODE_SOURCES = ("decode.cu", "ptx.cuh", "common.cuh", "merge.cuh", "quant.cuh")
+DECODE_SOURCES = ("decode.cu", "decode_split.cu", "decode_frag.cuh", "ptx.cuh", "common.cuh",
+                  "merge.cuh", "quant.cuh")
 PREFILL_SOURCES = ("prefill.cu", "ptx.cuh", "common.cuh")
 STREAM_METRIC = "q8_0/q4_0 host-streamed decode: H2D GB/s (% of measured H2D), query-tok/s at 262k ctx"
 

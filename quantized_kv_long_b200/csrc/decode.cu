@@ -50,12 +50,16 @@
 #include "merge.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "decode_frag.cuh"
 
 namespace kvq {
 
 bool launch_decode_simple(const DecodeArgs &a, cudaStream_t s);
+bool launch_decode_split(const DecodeArgs &a, cudaStream_t s);
 
 namespace {
+
+using namespace frag;
 
 constexpr int NPAIR = 6;                      // warp pairs per CTA
 constexpr int WARPS = 2 * NPAIR;
@@ -85,51 +89,6 @@ struct __align__(16) DecodeSmem {
 };
 // fused step: chunks whose merge weights fit in the ring, per 64-thread group
 constexpr int FUSED_SMEM_CHUNKS = (int)(NS * STAGE_BYTES / (NPAIR * sizeof(float)));
-
-// Four int8 in a u32 -> two half2 holding the exact integers:
-// (0x64 << 8 | (b ^ 0x80)) is the f16 1152 + b.
-__device__ __forceinline__ void s8x4_to_h2x2(uint32_t w, uint32_t &h01, uint32_t &h23)
-{
-    w ^= 0x80808080u;
-    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
-    h01 = ptx::h2_bits(__hsub2(ptx::bits_h2(ptx::prmt(w, 0x64646464u, 0x5140)), bias));
-    h23 = ptx::h2_bits(__hsub2(ptx::bits_h2(ptx::prmt(w, 0x64646464u, 0x7362)), bias));
-}
-
-// Nibbles at bits 0-3 and 16-19 of w -> half2 (u - 8); bits 4-7 and 20-23 -> half2 (u - 8).
-__device__ __forceinline__ uint32_t nib_lo(uint32_t w)
-{
-    const uint32_t x = (w & 0x000F000Fu) | 0x64006400u;  // 1024 + u
-    const __half2 c = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
-    return ptx::h2_bits(__hsub2(ptx::bits_h2(x), c));
-}
-
-__device__ __forceinline__ uint32_t nib_hi(uint32_t w)
-{
-    const uint32_t x = (w & 0x00F000F0u) | 0x64006400u;  // 1024 + 16u
-    const __half2 s = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
-    const __half2 c = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
-    return ptx::h2_bits(__hfma2(ptx::bits_h2(x), s, c));
-}
-
-__device__ __forceinline__ uint32_t lds16(const uint8_t *p)
-{
-    return *reinterpret_cast<const uint16_t *>(p);
-}
-
-__device__ __forceinline__ uint32_t lds32(const uint8_t *p)
-{
-    return *reinterpret_cast<const uint32_t *>(p);
-}
-
-// The four K bytes [p, p+4) of a k-step; 4-byte aligned exactly when `aligned`
-// (a constant once the block loop is unrolled).
-__device__ __forceinline__ uint32_t k_word(const uint8_t *p, bool aligned)
-{
-    if (aligned)
-        return lds32(p);
-    return ptx::prmt(lds16(p), lds16(p + 2), 0x5410);
-}
 
 template <int NT, bool FUSED>
 __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs a)
@@ -616,7 +575,7 @@ bool launch_decode(const DecodeArgs &a, cudaStream_t s)
             return launch_tc<1, true>(a, s);
         if (nt == 2)
             return launch_tc<2, true>(a, s);
-        return launch_tc<3, true>(a, s);
+        return launch_decode_split(a, s);
     }
     if (!a.force_simple && decode_tc_supported(a)) {
         const int rows = (a.n_q_heads / a.n_kv_heads) * a.T;
@@ -625,7 +584,7 @@ bool launch_decode(const DecodeArgs &a, cudaStream_t s)
             return launch_tc<1, false>(a, s);
         if (nt == 2)
             return launch_tc<2, false>(a, s);
-        return launch_tc<3, false>(a, s);
+        return launch_decode_split(a, s);  // three n-tiles: the role-split kernel
     }
     return launch_decode_simple(a, s);
 }
