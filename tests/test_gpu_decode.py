@@ -86,8 +86,11 @@ def test_fully_masked_last_chunk(kvq, T, kernel):
 
 
 @pytest.mark.parametrize("D,H,Hq,T", [(64, 2, 16, 2), (128, 8, 32, 1), (512, 1, 8, 4),
-                                      (256, 4, 4, 4), (32, 1, 1, 1), (256, 2, 16, 4)])
+                                      (256, 4, 4, 4), (32, 1, 1, 1), (256, 2, 16, 4),
+                                      (256, 2, 10, 4), (256, 1, 8, 3), (256, 3, 12, 4)])
 def test_other_shapes(kvq, D, H, Hq, T):
+    """Other head sizes and GQA groups; at head_dim 256, 20 and 24 rows (group 5 x 4
+    tokens, 8 x 3) take the role-split kernel and 16 rows (4 x 4) the pair kernel."""
     w = wl.small(wl.WORKLOADS["tiny"], head_dim=D, n_kv_heads=H, n_q_heads=Hq,
                  scale=float(D) ** -0.5)
     check_case(kvq, w, 2, T, 700, 128)
@@ -140,23 +143,25 @@ def test_tc_stage_edges(kvq, n_kv, chunk):
     check_case(kvq, w, 1, 1, n_kv, chunk)
 
 
-def test_bounded_wait_times_out_and_context_survives(kvq, monkeypatch):
+@pytest.mark.parametrize("T", [1, 4])
+def test_bounded_wait_times_out_and_context_survives(kvq, monkeypatch, T):
     """A wait on a barrier that nothing completes runs out after about a
     second: the kernel ends, kvq_check reports KVQ_ERR_TIMEOUT once, and the
-    next call on the same context is correct again."""
+    next call on the same context is correct again.  T = 1 runs the pair
+    kernel, T = 4 the role-split kernel."""
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=512)
     cache, orc = fill_both(w, [0], 512, 512)
-    q = q_all(w, [0], 4)
+    q = q_all(w, [0], T)
     monkeypatch.setenv("KVQ_TEST_DECODE_TIMEOUT", "1")
     qt = torch.from_numpy(q).cuda()
-    op = torch.empty((1, 4, 24, 1, 256), device="cuda")
-    lp = torch.empty((1, 4, 24, 1), device="cuda")
-    kvq.kvq_decode_attn(cache.layers(), qt, 24, 4, 512, 512, w.scale, op, lp)
+    op = torch.empty((1, T, 24, 1, 256), device="cuda")
+    lp = torch.empty((1, T, 24, 1), device="cuda")
+    kvq.kvq_decode_attn(cache.layers(), qt, 24, T, 512, 512, w.scale, op, lp)
     with pytest.raises(kvq.KvqError) as e:
         kvq.kvq_check()
     assert e.value.status == kvq.KVQ_ERR_TIMEOUT
     kvq.kvq_check()  # the status word was cleared
     monkeypatch.delenv("KVQ_TEST_DECODE_TIMEOUT")
-    op2, lp2, out, lse = run_decode(kvq, cache, q, 24, 4, 512, 512, w.scale)
+    op2, lp2, out, lse = run_decode(kvq, cache, q, 24, T, 512, 512, w.scale)
     rp, rl = oracle.decode_attn(orc[0][0], orc[0][1], q[0], 512, 512, w.scale)
     assert_attn_close(op2[0], lp2[0], rp, rl, "after timeout")
