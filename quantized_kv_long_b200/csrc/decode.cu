@@ -109,6 +109,18 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs 
     const uint8_t *kg = a.layers.k[layer] + ((int64_t)h * cap + c0) * KROW;
     const uint8_t *vg = a.layers.v[layer] + ((int64_t)h * cap + c0) * VROW;
 
+    // one stage's K and V rows into its ring slot (one thread; the slot is free)
+    auto copy_stage = [&](int st) {
+        const int slot = st % NS;
+        const int rows = min(TOK, n_tok - st * TOK);
+        ptx::mbar_arrive_expect_tx(&sm.full[slot], rows * (KROW + VROW));
+        ptx::bulk_g2s(sm.ring[slot], kg + (int64_t)st * STAGE_K, rows * KROW, &sm.full[slot]);
+        ptx::bulk_g2s(sm.ring[slot] + STAGE_K, vg + (int64_t)st * STAGE_V, rows * VROW,
+                      &sm.full[slot]);
+    };
+    // without an append to come first, the first stages are requested before anything
+    // else, so that their latency overlaps the set-up below
+    const int early = FUSED ? 0 : min(NS, n_stages);
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             ptx::mbar_init(&sm.full[i], 1);
@@ -117,6 +129,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs 
         ptx::mbar_init(&sm.never, 1);
         sm.abort = 0;
         ptx::fence_mbar_init();
+        for (int st = 0; st < early; ++st)
+            copy_stage(st);
     }
     // Q^T B-fragments: entry (hf, ks, nt, lane) holds q[row nt*8 + lane/4] dims
     // 128 hf + 16 ks + 4 (lane%4) .. +3 (the permuted k order; zero for padded rows)
@@ -177,14 +191,10 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs 
             (!ptx::mbar_wait_bounded(&sm.empty[slot], (round - 1) & 1, abort, WAIT_LIMIT_NS) ||
              !ptx::mbar_wait_bounded(&sm.full[slot], (round - 1) & 1, abort, WAIT_LIMIT_NS)))
             return false;
-        const int rows = min(TOK, n_tok - st * TOK);
-        ptx::mbar_arrive_expect_tx(&sm.full[slot], rows * (KROW + VROW));
-        ptx::bulk_g2s(sm.ring[slot], kg + (int64_t)st * STAGE_K, rows * KROW, &sm.full[slot]);
-        ptx::bulk_g2s(sm.ring[slot] + STAGE_K, vg + (int64_t)st * STAGE_V, rows * VROW,
-                      &sm.full[slot]);
+        copy_stage(st);
         return true;
     };
-    int issued = 0;
+    int issued = threadIdx.x == 0 ? early : 0;
     if (threadIdx.x == 0)
         for (; issued < NS && issued < n_stages; ++issued)
             issue(issued);

@@ -150,6 +150,18 @@ __global__ void __launch_bounds__(THREADS, 1) decode_split_kernel(const DecodeAr
     const uint8_t *kg = a.layers.k[layer] + ((int64_t)h * cap + c0) * KROW;
     const uint8_t *vg = a.layers.v[layer] + ((int64_t)h * cap + c0) * VROW;
 
+    // one stage's K and V rows into its ring slot (one thread; the slot is free)
+    auto copy_stage = [&](int st) {
+        const int slot = st % NS;
+        const int rows = min(TOK, n_tok - st * TOK);
+        ptx::mbar_arrive_expect_tx(&sm.full[slot], rows * (KROW + VROW));
+        ptx::bulk_g2s(sm.ring[slot], kg + (int64_t)st * STAGE_K, rows * KROW, &sm.full[slot]);
+        ptx::bulk_g2s(sm.ring[slot] + STAGE_K, vg + (int64_t)st * STAGE_V, rows * VROW,
+                      &sm.full[slot]);
+    };
+    // without an append to come first, the first stages are requested before anything
+    // else, so that their latency overlaps the set-up below
+    const int early = FUSED ? 0 : min(NS, n_stages);
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             ptx::mbar_init(&sm.full[i], 1);
@@ -162,6 +174,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_split_kernel(const DecodeAr
         ptx::mbar_init(&sm.never, 1);
         sm.abort = 0;
         ptx::fence_mbar_init();
+        for (int st = 0; st < early; ++st)
+            copy_stage(st);
     }
     // Q^T B-fragments: entry (ks, nt, lane) holds q[row nt*8 + lane/4] dims
     // 16 ks + 4 (lane%4) .. +3 (the permuted k order; zero for padded rows)
@@ -219,8 +233,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_split_kernel(const DecodeAr
     if (warp == PROD) {
         // ------------------------------------------------------------ copies
         if (lane == 0) {
-            int issued = 0;
-            for (int st = 0; st < n_stages; ++st) {
+            int issued = early;
+            for (int st = early; st < n_stages; ++st) {
                 const int slot = st % NS;
                 const uint32_t round = st / NS;
                 // refill once every warp released the slot and its previous copy landed
@@ -235,11 +249,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_split_kernel(const DecodeAr
                 }
                 if (*abort)
                     break;
-                const int rows = min(TOK, n_tok - st * TOK);
-                ptx::mbar_arrive_expect_tx(&sm.full[slot], rows * (KROW + VROW));
-                ptx::bulk_g2s(sm.ring[slot], kg + (int64_t)st * STAGE_K, rows * KROW, &sm.full[slot]);
-                ptx::bulk_g2s(sm.ring[slot] + STAGE_K, vg + (int64_t)st * STAGE_V, rows * VROW,
-                              &sm.full[slot]);
+                copy_stage(st);
                 ++issued;
             }
             // drain: every issued copy has landed before the ring is reused or freed
