@@ -159,9 +159,10 @@ __global__ void __launch_bounds__(THREADS, 1) decode_split_kernel(const DecodeAr
         ptx::bulk_g2s(sm.ring[slot] + STAGE_K, vg + (int64_t)st * STAGE_V, rows * VROW,
                       &sm.full[slot]);
     };
-    // without an append to come first, the first stages are requested before anything
-    // else, so that their latency overlaps the set-up below
-    const int early = FUSED ? 0 : min(NS, n_stages);
+    // unless this chunk holds rows that the fused step appends first, the first stages
+    // are requested before anything else, so that their latency overlaps the set-up
+    const bool appends_here = FUSED && c0 + n_tok > a.n_kv - a.T;
+    const int early = appends_here ? 0 : min(NS, n_stages);
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             ptx::mbar_init(&sm.full[i], 1);
