@@ -98,7 +98,7 @@ typedef void *kvq_stream;
  * for V.  All layers passed to one call must use the same formats.  Append,
  * the general decode path (kvq_decode_attn, kvq_decode_step,
  * kvq_decode_merged_static, kvq_stream_decode) accept every combination; the
- * tiled decode kernel, the fused step's single launch and kvq_prefill_attn
+ * tiled decode kernels, the fused step's single launch and kvq_prefill_attn
  * implement the default pair only (decode falls back to the general kernel,
  * the step to three launches, prefill returns KVQ_ERR_UNSUPPORTED). */
 typedef enum kvq_type {
@@ -230,7 +230,7 @@ kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t r
  *                cleared by the call itself (a cudaMemsetAsync on `stream`
  *                before the kernel); owned by the caller, not used after the
  *                step completes
- * Shapes outside the tiled decode kernel (head_dim != 256, or more than 24
+ * Shapes outside the tiled decode kernels (head_dim != 256, or more than 24
  * rows per KV head) run the same step as three launches (append, decode,
  * merge).
  * Errors: those of kvq_append, kvq_decode_attn and kvq_merge_lse; WORKSPACE

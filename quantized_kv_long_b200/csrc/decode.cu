@@ -11,7 +11,8 @@
 // lse = m + ln l.
 //
 // Layout of the work (head_dim 256, up to 24 rows = G*T):
-//  * one CTA per (layer, KV head, chunk) of NPAIR warp pairs; thread 0 also
+//  * one CTA per (layer, KV head, chunk) of NPAIR warp pairs (8 for up to 8
+//    rows, 6 for up to 16: PairCfg); thread 0 also
 //    issues the copies: a prologue of NS stages, then each stage's slot is
 //    refilled as soon as every warp has released it;
 //  * the chunk streams in stages of 16*NPAIR tokens -- that many K head-rows
@@ -61,15 +62,22 @@ namespace {
 
 using namespace frag;
 
-constexpr int NPAIR = 6;                      // warp pairs per CTA
-constexpr int WARPS = 2 * NPAIR;
-constexpr int THREADS = 32 * WARPS;
-constexpr int TOK = 16 * NPAIR;               // tokens per stage
-constexpr int NS = 4;                         // stages in the ring
 constexpr int KROW = 272, VROW = 144;         // head-row bytes at head_dim 256
-constexpr int STAGE_K = TOK * KROW;
-constexpr int STAGE_V = TOK * VROW;
-constexpr int STAGE_BYTES = STAGE_K + STAGE_V;
+// Launch shape per number of n-tiles of rows: with one n-tile (up to 8 rows) a
+// warp's O^T takes 32 registers, so 8 warp pairs fit the register file (and a
+// 3-stage ring of 128-token stages the shared memory); with two, 6 pairs and a
+// 4-stage ring of 96-token stages.
+template <int NT>
+struct PairCfg {
+    static constexpr int NPAIR = NT == 1 ? 8 : 6;  // warp pairs per CTA
+    static constexpr int WARPS = 2 * NPAIR;
+    static constexpr int THREADS = 32 * WARPS;
+    static constexpr int TOK = 16 * NPAIR;         // tokens per stage
+    static constexpr int NS = NT == 1 ? 3 : 4;     // stages in the ring
+    static constexpr int STAGE_K = TOK * KROW;
+    static constexpr int STAGE_V = TOK * VROW;
+    static constexpr int STAGE_BYTES = STAGE_K + STAGE_V;
+};
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
@@ -78,21 +86,26 @@ constexpr float M_INIT = -1.0e30f;            // "no score yet", finite: ex2(s -
 
 template <int NT>
 struct __align__(16) DecodeSmem {
-    uint8_t ring[NS][STAGE_BYTES];
-    float4 xs[NPAIR][2][2][NT][32];  // partial S exchange [pair][parity][half][n-tile][lane]
-    uint2 qf[2][8][NT][32];          // Q^T B-fragments [half][k-step][n-tile][lane]
-    float pm[NPAIR][32], pl[NPAIR][32];
-    float red[NPAIR][2];  // fused step: per-group reduction slots of the merge
-    uint64_t full[NS], empty[NS], never;
+    using C = PairCfg<NT>;
+    uint8_t ring[C::NS][C::STAGE_BYTES];
+    float4 xs[C::NPAIR][2][2][NT][32];  // partial S exchange [pair][parity][half][n-tile][lane]
+    uint2 qf[2][8][NT][32];             // Q^T B-fragments [half][k-step][n-tile][lane]
+    float pm[C::NPAIR][32], pl[C::NPAIR][32];
+    float red[C::NPAIR][2];  // fused step: per-group reduction slots of the merge
+    uint64_t full[C::NS], empty[C::NS], never;
     int abort;
     int last;             // fused step: this CTA is the last of its (layer, KV head)
 };
-// fused step: chunks whose merge weights fit in the ring, per 64-thread group
-constexpr int FUSED_SMEM_CHUNKS = (int)(NS * STAGE_BYTES / (NPAIR * sizeof(float)));
 
 template <int NT, bool FUSED>
-__global__ void __launch_bounds__(THREADS, 1) decode_tc_kernel(const DecodeArgs a)
+__global__ void __launch_bounds__(PairCfg<NT>::THREADS, 1) decode_tc_kernel(const DecodeArgs a)
 {
+    using Cfg = PairCfg<NT>;
+    constexpr int NPAIR = Cfg::NPAIR, WARPS = Cfg::WARPS, THREADS = Cfg::THREADS, TOK = Cfg::TOK,
+                  NS = Cfg::NS, STAGE_K = Cfg::STAGE_K, STAGE_V = Cfg::STAGE_V,
+                  STAGE_BYTES = Cfg::STAGE_BYTES;
+    // fused step: chunks whose merge weights fit in the ring, per 64-thread group
+    constexpr int FUSED_SMEM_CHUNKS = (int)(NS * STAGE_BYTES / (NPAIR * sizeof(float)));
     extern __shared__ __align__(128) uint8_t smem_raw[];
     DecodeSmem<NT> &sm = *reinterpret_cast<DecodeSmem<NT> *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -563,7 +576,7 @@ bool launch_tc(const DecodeArgs &a, cudaStream_t s)
     const int64_t grid = (int64_t)a.n_layers * a.n_kv_heads * C;
     if (grid >= (1ll << 31))
         return false;
-    decode_tc_kernel<NT, FUSED><<<(unsigned)grid, THREADS, smem, s>>>(a);
+    decode_tc_kernel<NT, FUSED><<<(unsigned)grid, PairCfg<NT>::THREADS, smem, s>>>(a);
     return true;
 }
 
