@@ -4,7 +4,8 @@ Expected values come from closed forms (one key, identical keys, zero query),
 from a library routine (torch's fp64 scaled_dot_product_attention and
 logsumexp on CPU over the oracle's pinned dequantization), or from invariants
 of the method (chunked merge = one pass, merge associativity, fully masked
-chunk is a no-op, prefill row = decode of that token).
+chunk is a no-op, a uniform logit shift moves only the lse, prefill row =
+decode of that token).
 """
 import math
 
@@ -68,6 +69,38 @@ def test_identical_keys_give_mean_value_and_log_count():
         assert np.allclose(out[0, g, 0], V[0, :n].mean(axis=0), rtol=0, atol=1e-12)
         s = SCALE * float(np.dot(q[0, g].astype(np.float64), K[0, 0]))
         assert abs(lse[0, g, 0] - (s + math.log(n))) < 1e-12
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_uniform_logit_shift_moves_lse_only(T):
+    """Softmax invariance: adding the same constant to every logit of a row leaves
+    its output unchanged and adds the constant to its lse.  Every key gets the same
+    first 32-element block (so the same dequantized values there); a query that
+    differs only in that block shifts all of a row's logits by
+    scale * dq . k_block0, computed here in fp64 from the pinned dequantization."""
+    H, D, n = 2, 64, 150
+    rng = np.random.default_rng(7)
+    k = rng.standard_normal((n, H, D)).astype(np.float32)
+    v = rng.standard_normal((n, H, D)).astype(np.float32)
+    k[:, :, 32:36] *= 8
+    k[:, :, :32] = k[0, :, :32]
+    kc, vc = oracle.empty_cache(H, D, n)
+    oracle.append(kc, vc, k, v, 0)
+    K, _ = _deq(kc, vc)
+    assert np.array_equal(K[:, 0, :32], K[:, n - 1, :32])
+    q = _q(T, 4, D, 8)
+    q2 = q.copy()
+    dq = (np.random.default_rng(9).standard_normal((T, 4, 32)) * 2).astype(np.float16)
+    q2[:, :, :32] = dq
+    o1, l1 = oracle.decode_attn(kc, vc, q, n_kv=n, chunk=n, scale=SCALE)
+    o2, l2 = oracle.decode_attn(kc, vc, q2, n_kv=n, chunk=n, scale=SCALE)
+    for t in range(T):
+        for g in range(4):
+            h = g // 2
+            shift = SCALE * float(np.dot(q2[t, g, :32].astype(np.float64) -
+                                         q[t, g, :32].astype(np.float64), K[h, 0, :32]))
+            assert np.allclose(o2[t, g, 0], o1[t, g, 0], rtol=0, atol=1e-12)
+            assert abs(l2[t, g, 0] - (l1[t, g, 0] + shift)) < 1e-10
 
 
 @pytest.mark.parametrize("T", [1, 4])
