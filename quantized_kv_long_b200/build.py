@@ -22,7 +22,10 @@ COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler",
           "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
 # The quantizers are a sequence of separately rounded fp32 operations: no FMA
 # contraction anywhere in that file (they also use explicit __f*_rn intrinsics).
-PER_FILE = {"quant.cu": ["-fmad=false"]}
+# The persistent decode kernel sets per-warpgroup register budgets (setmaxnreg);
+# a spill inside such a region is refused at build time.
+PER_FILE = {"quant.cu": ["-fmad=false"],
+            "decode_tmem.cu": ["-Xptxas", "--warn-on-spills", "-Xptxas", "--warning-as-error"]}
 
 
 def nvcc() -> str:

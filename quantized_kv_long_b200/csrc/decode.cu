@@ -57,6 +57,7 @@ namespace kvq {
 
 bool launch_decode_simple(const DecodeArgs &a, cudaStream_t s);
 bool launch_decode_split(const DecodeArgs &a, cudaStream_t s);
+bool launch_decode_tmem(const DecodeArgs &a, cudaStream_t s);
 
 namespace {
 
@@ -601,15 +602,8 @@ bool launch_decode(const DecodeArgs &a, cudaStream_t s)
             return launch_tc<2, true>(a, s);
         return launch_decode_split(a, s);
     }
-    if (!a.force_simple && decode_tc_supported(a)) {
-        const int rows = (a.n_q_heads / a.n_kv_heads) * a.T;
-        const int nt = (rows + 7) / 8;
-        if (nt == 1)
-            return launch_tc<1, false>(a, s);
-        if (nt == 2)
-            return launch_tc<2, false>(a, s);
-        return launch_decode_split(a, s);  // three n-tiles: the role-split kernel
-    }
+    if (!a.force_simple && decode_tc_supported(a))
+        return launch_decode_tmem(a, s);
     return launch_decode_simple(a, s);
 }
 
