@@ -220,26 +220,17 @@ def run_ours(args, w: wl.Workload) -> dict | None:
 
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
-    ws = torch.empty(kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE_STEP, L, Hq, w.n_kv_heads, T, D),
-                     dtype=torch.uint8, device=device)
 
     def step(i=None):
-        if not args.fused:  # append, decode, merge as three launches
-            kvq.kvq_append(layers, k_new, v_new, n_kv - T, T, stream)
-            if i is not None:
-                ev_dec[i][0].record(stream)
-            kvq.kvq_decode_attn(layers, q, Hq, T, n_kv, chunk, w.scale, op, lp, stream)
-            if i is not None:
-                ev_dec[i][1].record(stream)
-            kvq.kvq_merge_lse(op, lp, rows, C, D, out, lse, stream)
-            return
-        # one launch (after clearing its per-head counters): append + decode + merge
+        # append, decode, merge: the three launches of kvq_decode_step, issued one by one
+        # so that the decode launch can be timed on its own
+        kvq.kvq_append(layers, k_new, v_new, n_kv - T, T, stream)
         if i is not None:
             ev_dec[i][0].record(stream)
-        kvq.kvq_decode_step(layers, k_new, v_new, q, Hq, T, n_kv, chunk, w.scale, op, lp, out,
-                            lse, ws, stream=stream)
+        kvq.kvq_decode_attn(layers, q, Hq, T, n_kv, chunk, w.scale, op, lp, stream)
         if i is not None:
             ev_dec[i][1].record(stream)
+        kvq.kvq_merge_lse(op, lp, rows, C, D, out, lse, stream)
 
     for _ in range(args.warmup):
         step()
@@ -303,8 +294,6 @@ def run_ours(args, w: wl.Workload) -> dict | None:
         gbs = weak_gbs(world, kv_bytes, ms)
         achieved = kv_bytes / (dec_ms_max * 1e-3) / 1e9
         tr = traffic_record(DECODE_SOURCES)
-        if tr is not None and bool(tr.get("fused", False)) != args.fused:
-            tr = None  # the record is of the other launch sequence
         res = {
             "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
@@ -314,8 +303,7 @@ def run_ours(args, w: wl.Workload) -> dict | None:
                        "head_dim": D, "context": n_kv, "query_tokens": T, "chunk": chunk,
                        "seed": w.seed, "kv_bytes_per_step": kv_bytes,
                        "l2": "inputs larger than L2 (7 GB cache vs 126 MB)",
-                       "step": ("append, decode, merge: 3 launches" if not args.fused else
-                                "kvq_decode_step: 1 launch (+ a 256-byte memset)"),
+                       "step": "append, decode, merge: 3 launches",
                        "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
             # query tokens per step (each attends all L layers) / step time
             "query_tok_per_s": round(world * T / (ms * 1e-3), 1),
@@ -325,14 +313,12 @@ def run_ours(args, w: wl.Workload) -> dict | None:
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 4)},
             "roofline": {"bound": "hbm",
-                         "kernel": ("kvq_decode_attn (16 layers, 1 launch)" if not args.fused else
-                                    "kvq_decode_step: append + decode + merge of 16 layers, "
-                                    "1 launch"),
+                         "kernel": f"kvq_decode_attn ({L} layers, 1 launch)",
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": tr["dram_bytes_per_launch"] if tr else None,
                          "launch_ms": round(dec_ms_max, 4)},
-            "gpu_launches": (1 if args.fused else 3) * args.steps,
+            "gpu_launches": 3 * args.steps,
             "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
                        "reasons": cl["reasons"], "samples": cl["samples"]},
         }
@@ -342,7 +328,7 @@ def run_ours(args, w: wl.Workload) -> dict | None:
     return res
 
 
-DECODE_SOURCES = ("decode.cu", "decode_tmem.cu", "decode_split.cu", "decode_frag.cuh", "ptx.cuh", "common.cuh",
+DECODE_SOURCES = ("decode.cu", "decode_tmem.cu", "decode_frag.cuh", "ptx.cuh", "common.cuh",
                   "merge.cuh", "quant.cuh")
 PREFILL_SOURCES = ("prefill.cu", "ptx.cuh", "common.cuh")
 STREAM_METRIC = "q8_0/q4_0 host-streamed decode: H2D GB/s (% of measured H2D), query-tok/s at 262k ctx"
@@ -663,9 +649,6 @@ def main(argv=None) -> int:
     ap.add_argument("--budget-mib", type=int, default=None,
                     help="stream262k: device memory for the cache; the layers that fit next to "
                          "the two streaming slots stay resident (default: all streamed)")
-    ap.add_argument("--fused", action="store_true",
-                    help="decode configs: time the step as one kvq_decode_step launch "
-                         "(default: append, decode and merge as three launches)")
     ap.add_argument("--layers", type=int, default=None,
                     help="profile a smaller case of the same kernel: only this many layers")
     args = ap.parse_args(argv)

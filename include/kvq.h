@@ -210,31 +210,23 @@ kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t r
 /* Fused decode step                                                       */
 /* ---------------------------------------------------------------------- */
 
-/* One decode step of all layers in one kernel launch:
+/* One decode step of all layers:
  *   kvq_append(layers, k_new, v_new, pos = n_kv - T, T), then
  *   kvq_decode_attn(...), then kvq_merge_lse(...)
- * with the same results (cache bytes, out_part, lse_part, out, lse) as those
- * three calls.  Inside the launch, the CTA whose chunk holds a new row
- * quantizes it before reading the chunk, and the last CTA of each
- * (layer, KV head) to finish merges that head's chunk partials while they
- * are still in L2; the merge kernel's launch and its re-read of the partials
- * from memory go away.  Source: the ROCm adaptive KV-streaming page, the
- * paragraph on the fork's RDNA kernel work (single-queue async graphs,
- * persistent graph arenas): a decode step as one queue submission.
+ * issued as those three launches, back to back on `stream`, with the same
+ * results (cache bytes, out_part, lse_part, out, lse).  All arguments are
+ * checked before the first launch.  A single launch that appends in the
+ * decode kernel and merges in the last CTA of each head was built and
+ * measured: it saved two launches of a few microseconds on a step of
+ * milliseconds and cost more inside the decode kernel than that, so the step
+ * is three launches (capture them in a CUDA graph to drop the launch gaps).
  *  k_new, v_new  device fp32 [n_layers][T][n_kv_heads][head_dim], 16-B aligned
  *  n_kv          keys after the append (the new rows are [n_kv - T, n_kv))
  *  q, out_part, lse_part, out, lse, chunk, scale: as kvq_decode_attn and
  *                kvq_merge_lse (rows = n_layers * T * n_q_heads)
- *  workspace     device, 4-B aligned, >= kvq_workspace_bytes(KVQ_OP_DECODE_STEP,
- *                ...) = n_layers * n_kv_heads * 4 bytes: per-head counters,
- *                cleared by the call itself (a cudaMemsetAsync on `stream`
- *                before the kernel); owned by the caller, not used after the
- *                step completes
- * Shapes outside the tiled decode kernels (head_dim != 256, or more than 24
- * rows per KV head) run the same step as three launches (append, decode,
- * merge).
- * Errors: those of kvq_append, kvq_decode_attn and kvq_merge_lse; WORKSPACE
- *         (null, too small or misaligned workspace). */
+ *  workspace, ws_bytes  reserved: not read; may be NULL / 0
+ *                (kvq_workspace_bytes(KVQ_OP_DECODE_STEP, ...) is 0)
+ * Errors: those of kvq_append, kvq_decode_attn and kvq_merge_lse. */
 kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k_new,
                            const float *v_new, const uint16_t *q, int n_q_heads, int T,
                            int64_t n_kv, int chunk, float scale, float *out_part,
@@ -265,8 +257,14 @@ kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k
  *  page      keys per page, a positive multiple of 128 (the online merge makes
  *            the result independent of it)
  *  out, lse  device fp32 [n_layers][T][n_q_heads][head_dim] and [...][n_q_heads]
- *  page_out, page_lse  must be NULL: per-page partial outputs are not built
- *            (both set -> KVQ_ERR_UNSUPPORTED)
+ *  page_out, page_lse  optional (both NULL or both set), device fp32
+ *            [n_layers][T][n_q_heads][n_pages][head_dim] (16-B aligned) and
+ *            [n_layers][T][n_q_heads][n_pages], n_pages = ceil((n_cached + T) /
+ *            page): the partial of page p (keys [p page, (p + 1) page) that the
+ *            row sees) as out = sum_j p_j v^_j / l and lse = m + ln l, out = 0 and
+ *            lse = -inf where the row sees no key of the page.  out and lse are
+ *            then the LSE merge of the pages (the kvq_merge_lse kernel, launched
+ *            by this call after the prefill kernels).
  *  workspace optional, device, 256-B aligned.  NULL: each CTA of the
  *            tensor-core path dequantizes the key tiles it reads.  Otherwise
  *            ws_bytes >= kvq_prefill_workspace_bytes(n_layers, n_kv_heads,
@@ -277,9 +275,9 @@ kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k
  *            keys).  Same results bit for bit.  Ignored when the tensor-core
  *            path does not run.  Owned by the caller; not used after the call's
  *            work completes.
- * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (group size > 32, page outputs,
- *         block formats other than Q8_0 K / Q4_0 V), WORKSPACE (a workspace
- *         smaller than needed), CUDA. */
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (group size > 32, block formats
+ *         other than Q8_0 K / Q4_0 V), WORKSPACE (a workspace smaller than
+ *         needed), CUDA. */
 kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
                             int n_q_heads, int T, int64_t n_cached, int page, float scale,
                             float *out, float *lse, float *page_out, float *page_lse,
@@ -382,9 +380,10 @@ size_t kvq_prefill_workspace_bytes(int n_layers, int n_kv_heads, int head_dim, i
 #define KVQ_OP_PREFILL 2
 #define KVQ_OP_DECODE_STEP 3
 
-/* Bytes of device workspace an operation needs (0 if none).
- * KVQ_OP_DECODE: always 0.  KVQ_OP_PREFILL: n_layers, n_q_heads, T as the call.
- * KVQ_OP_DECODE_STEP: n_layers * n_kv_heads * 4.
+/* Bytes of device workspace an operation requires (0 if none).
+ * KVQ_OP_DECODE: always 0.  KVQ_OP_PREFILL: always 0 -- its workspace is
+ * optional and its size depends on the key count, see
+ * kvq_prefill_workspace_bytes.  KVQ_OP_DECODE_STEP: always 0.
  * Returns (size_t)-1 for an unknown op. */
 size_t kvq_workspace_bytes(int op, int n_layers, int n_q_heads, int n_kv_heads, int T,
                            int head_dim);
@@ -402,6 +401,31 @@ const char *kvq_last_error(void);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int kvq_version(void);
+
+/* ---------------------------------------------------------------------- */
+/* Test hooks                                                              */
+/* ---------------------------------------------------------------------- */
+
+/* Process-wide switches for the library's own tests (all off by default; no
+ * production caller sets them).  Each call reads them once (atomic loads); the
+ * library reads no environment variables.
+ *  decode_general     1: decode runs on the general kernel (kernel comparisons)
+ *  decode_timeout     1: every decode launch waits on a barrier that nothing
+ *                     completes, so its bounded wait runs out (about a second)
+ *                     and kvq_check reports KVQ_ERR_TIMEOUT
+ *  prefill_timeout    1: the same for the tensor-core prefill launches (the
+ *                     tile expansion and the attention kernel)
+ *  stream_fail_layer  >= 0: kvq_stream_decode fails the host-to-device copy of
+ *                     this layer (a host-side injected fault); -1: off */
+typedef struct kvq_test_hooks {
+    int32_t decode_general;
+    int32_t decode_timeout;
+    int32_t prefill_timeout;
+    int32_t stream_fail_layer;
+} kvq_test_hooks;
+
+/* Set the test hooks; NULL turns them all off.  Always KVQ_OK. */
+kvq_status kvq_test_set_hooks(const kvq_test_hooks *hooks);
 
 #ifdef __cplusplus
 }

@@ -41,20 +41,29 @@ kvq_status check_launch(const char *what)
 
 kvq_status status_word(unsigned int **out)
 {
-    constexpr int MAX_DEV = 64;
-    static unsigned int *cache[MAX_DEV] = {};
+    // one entry per device; two threads that look the address up at the same time
+    // store the same value
+    static std::atomic<unsigned int *> cache[MAX_DEVICES];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV)
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
         return set_error(KVQ_ERR_CUDA, "no current CUDA device");
-    if (!cache[dev]) {
+    unsigned int *w = cache[dev].load(std::memory_order_acquire);
+    if (!w) {
         void *p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
         if (e != cudaSuccess)
             return set_error(KVQ_ERR_CUDA, "status word: %s", cudaGetErrorString(e));
-        cache[dev] = static_cast<unsigned int *>(p);
+        w = static_cast<unsigned int *>(p);
+        cache[dev].store(w, std::memory_order_release);
     }
-    *out = cache[dev];
+    *out = w;
     return KVQ_OK;
+}
+
+TestHooks &test_hooks()
+{
+    static TestHooks h;
+    return h;
 }
 
 // ---- validation helpers ---------------------------------------------------
@@ -176,11 +185,9 @@ static kvq_status fill_decode(const kvq_layer *layers, int n_layers, const uint1
     a.out_part = out_part;
     a.lse_part = lse_part;
     KVQ_TRY(status_word(&a.status));
-    // host-side test hooks (environment): the general kernel, a forced wait timeout
-    const char *ks = getenv("KVQ_DECODE_KERNEL");
-    a.force_simple = ks && strcmp(ks, "simple") == 0;
-    const char *tt = getenv("KVQ_TEST_DECODE_TIMEOUT");
-    a.test_timeout = tt && atoi(tt) != 0;
+    // test hooks (kvq_test_set_hooks): the general kernel, a forced wait timeout
+    a.force_simple = test_hooks().decode_general.load(std::memory_order_relaxed);
+    a.test_timeout = test_hooks().decode_timeout.load(std::memory_order_relaxed);
     return KVQ_OK;
 }
 
@@ -305,40 +312,21 @@ kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k
                            float *lse_part, float *out, float *lse, void *workspace,
                            size_t ws_bytes, kvq_stream stream)
 {
+    (void)workspace;  // reserved: the step needs none
+    (void)ws_bytes;
     const char *fn = "kvq_decode_step";
     KVQ_TRY(validate_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
                             lse_part, fn));
     KVQ_TRY(need(k_new, 16, "k_new", fn));
     KVQ_TRY(need(v_new, 16, "v_new", fn));
-    const int H = layers[0].n_kv_heads, D = layers[0].head_dim;
+    const int D = layers[0].head_dim;
     const int64_t rows = (int64_t)n_layers * T * n_q_heads;
     const int n_chunks = (int)((n_kv + chunk - 1) / chunk);
     KVQ_TRY(validate_merge(out_part, lse_part, rows, n_chunks, D, out, lse, fn));
-    const size_t ws_need = kvq_workspace_bytes(KVQ_OP_DECODE_STEP, n_layers, n_q_heads, H, T, D);
-    if (!workspace || ws_bytes < ws_need || !aligned(workspace, 4))
-        return set_error(KVQ_ERR_WORKSPACE,
-                         "%s: needs a 4-byte aligned workspace of %zu bytes (got %zu at %p)", fn,
-                         ws_need, ws_bytes, workspace);
-    const cudaStream_t s = as_stream(stream);
     DecodeArgs a;
     KVQ_TRY(fill_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
                         lse_part, a));
-    if (!a.force_simple && decode_tc_supported(a)) {
-        // one launch: append, decode, and the merge in the last CTA of each (layer, KV head)
-        const cudaError_t e = cudaMemsetAsync(workspace, 0, ws_need, s);
-        if (e != cudaSuccess)
-            return set_error(KVQ_ERR_CUDA, "%s: clearing the workspace: %s", fn,
-                             cudaGetErrorString(e));
-        a.k_new = k_new;
-        a.v_new = v_new;
-        a.out = out;
-        a.lse = lse;
-        a.counters = static_cast<unsigned int *>(workspace);
-        if (!launch_decode(a, s))
-            return set_error(KVQ_ERR_UNSUPPORTED, "%s: no fused kernel for this shape", fn);
-        return check_launch(fn);
-    }
-    // other shapes: the same step as three launches
+    const cudaStream_t s = as_stream(stream);
     KVQ_TRY(kvq_append(layers, n_layers, k_new, v_new, n_kv - T, T, stream));
     if (!launch_decode(a, s))
         return set_error(KVQ_ERR_UNSUPPORTED, "%s: no kernel for this shape", fn);
@@ -363,7 +351,6 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
     if (page_out) {
         KVQ_TRY(need(page_out, 16, "page_out", fn));
         KVQ_TRY(need(page_lse, 4, "page_lse", fn));
-        return set_error(KVQ_ERR_UNSUPPORTED, "%s: per-page partial outputs are not built", fn);
     }
     const int H = layers[0].n_kv_heads, D = layers[0].head_dim;
     if (n_q_heads < 1 || n_q_heads % H != 0)
@@ -424,8 +411,17 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
         a.ws_bytes = ws_bytes;
     }
     KVQ_TRY(status_word(&a.status));
+    a.test_timeout = test_hooks().prefill_timeout.load(std::memory_order_relaxed);
     launch_prefill(a, as_stream(stream));
-    return check_launch(fn);
+    KVQ_TRY(check_launch(fn));
+    if (page_out) {
+        // the kernels wrote the per-page partials; out and lse are their merge
+        const int64_t rows = (int64_t)n_layers * T * n_q_heads;
+        const int n_pages = (int)((n_cached + T + page - 1) / page);
+        launch_merge_lse(page_out, page_lse, rows, n_pages, D, out, lse, as_stream(stream));
+        KVQ_TRY(check_launch(fn));
+    }
+    return KVQ_OK;
 }
 
 size_t kvq_prefill_workspace_bytes(int n_layers, int n_kv_heads, int head_dim, int64_t n_keys)
@@ -439,11 +435,9 @@ size_t kvq_workspace_bytes(int op, int n_layers, int n_q_heads, int n_kv_heads, 
     if (op == KVQ_OP_DECODE)
         return 0;
     if (op == KVQ_OP_DECODE_STEP)
-        return (n_layers > 0 && n_kv_heads > 0)
-                   ? (size_t)n_layers * n_kv_heads * sizeof(unsigned int)
-                   : (size_t)-1;
+        return 0;
     if (op == KVQ_OP_PREFILL)
-        return prefill_workspace_bytes(n_layers, n_q_heads, n_kv_heads, T, head_dim);
+        return 0;  // required: none (the optional workspace: kvq_prefill_workspace_bytes)
     return (size_t)-1;
 }
 
@@ -485,5 +479,15 @@ const char *kvq_status_string(kvq_status s)
 const char *kvq_last_error(void) { return t_err; }
 
 int kvq_version(void) { return 100; }
+
+kvq_status kvq_test_set_hooks(const kvq_test_hooks *hooks)
+{
+    TestHooks &h = test_hooks();
+    h.decode_general.store(hooks ? hooks->decode_general : 0);
+    h.decode_timeout.store(hooks ? hooks->decode_timeout : 0);
+    h.prefill_timeout.store(hooks ? hooks->prefill_timeout : 0);
+    h.stream_fail_layer.store(hooks ? hooks->stream_fail_layer : -1);
+    return KVQ_OK;
+}
 
 }  // extern "C"

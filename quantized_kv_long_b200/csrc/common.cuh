@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "kvq.h"
 
 namespace kvq {
@@ -47,10 +49,40 @@ __device__ __forceinline__ void report_timeout(unsigned int *status)
 // Bounded spin limit for any device-side wait (iterations of a try_wait loop).
 constexpr long long SPIN_LIMIT = 1ll << 26;
 
+// ---- test hooks (host): set only through kvq_test_set_hooks -------------------
+struct TestHooks {
+    std::atomic<int> decode_general{0}, decode_timeout{0}, prefill_timeout{0},
+        stream_fail_layer{-1};
+};
+TestHooks &test_hooks();
+
 // ---- error plumbing (host) ------------------------------------------------
 kvq_status set_error(kvq_status s, const char *fmt, ...);
 kvq_status check_launch(const char *what);
 kvq_status status_word(unsigned int **out);  // address of the current device's word
+
+// Dynamic shared memory limit of a kernel: raises it on the current device to at
+// least `bytes`, remembering the largest value set per device in `done` (one
+// array per kernel); safe to call from several host threads.
+constexpr int MAX_DEVICES = 64;
+inline bool ensure_smem(const void *kernel, std::atomic<int> (&done)[MAX_DEVICES], int bytes)
+{
+    if (bytes <= 48 * 1024)
+        return true;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
+        return false;
+    if (done[dev].load(std::memory_order_acquire) >= bytes)
+        return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return false;
+    int seen = done[dev].load(std::memory_order_relaxed);
+    while (seen < bytes && !done[dev].compare_exchange_weak(seen, bytes, std::memory_order_release))
+    {
+    }
+    return true;
+}
 
 inline bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 inline cudaStream_t as_stream(kvq_stream s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -76,16 +108,10 @@ struct DecodeArgs {
     unsigned int *status;  // device status word (bounded waits that ran out)
     int force_simple;      // host test hook: use the general kernel
     int test_timeout;      // host test hook: make the first wait run out
-    // fused step (all null otherwise): append k_new / v_new [layer][T][kv head][head_dim]
-    // at rows [n_kv - T, n_kv) first, and merge the chunk partials of each (layer, kv head)
-    // into out / lse in the last CTA of that head (counters: one zeroed int per head)
-    const float *k_new, *v_new;
-    float *out, *lse;
-    unsigned int *counters;
 };
 // Returns false (and launches nothing) if no kernel supports the shape.
 bool launch_decode(const DecodeArgs &a, cudaStream_t s);
-// The fused step (DecodeArgs::counters set) exists for the shapes of the tiled kernel.
+// True for the shapes of the persistent tensor-core kernel.
 bool decode_tc_supported(const DecodeArgs &a);
 
 struct PrefillArgs {
@@ -99,6 +125,7 @@ struct PrefillArgs {
     void *workspace;
     size_t ws_bytes;
     unsigned int *status;
+    int test_timeout;  // test hook: one bounded wait of each tensor-core launch runs out
 };
 size_t prefill_workspace_bytes(int n_layers, int n_q_heads, int n_kv_heads, int T, int head_dim);
 // Optional workspace of the tensor-core path: the f16 key tiles expanded once per

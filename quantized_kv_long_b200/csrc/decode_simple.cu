@@ -159,9 +159,9 @@ size_t decode_simple_smem(int R, int D)
 template <int KT, int VT>
 static bool launch_simple_typed(const DecodeArgs &a, size_t smem, cudaStream_t s)
 {
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(decode_simple_kernel<KT, VT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    static std::atomic<int> smem_set[MAX_DEVICES];
+    if (!ensure_smem(reinterpret_cast<const void *>(decode_simple_kernel<KT, VT>), smem_set,
+                     (int)smem))
         return false;
     const int n_chunks = (int)((a.n_kv + a.chunk - 1) / a.chunk);
     dim3 grid(n_chunks, a.n_kv_heads, a.n_layers);

@@ -931,21 +931,18 @@ __global__ void __launch_bounds__(THREADS, 1) decode_tmem_kernel(const DecodeArg
 }
 
 // Per-device one-time launch set-up: the shared-memory attribute and the SM count.
-std::atomic<int> g_sms[64];
+std::atomic<int> g_sms[MAX_DEVICES];
 
 template <int NT>
 bool launch_nt(const DecodeArgs &a, cudaStream_t s)
 {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
         return false;
-    static std::atomic<bool> attr_set[64];
-    if (!attr_set[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(decode_tmem_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem_bytes<NT>()) != cudaSuccess)
-            return false;
-        attr_set[dev].store(true, std::memory_order_release);
-    }
+    static std::atomic<int> smem_set[MAX_DEVICES];
+    if (!ensure_smem(reinterpret_cast<const void *>(decode_tmem_kernel<NT>), smem_set,
+                     smem_bytes<NT>()))
+        return false;
     int sms = g_sms[dev].load(std::memory_order_acquire);
     if (sms == 0) {
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
@@ -964,8 +961,8 @@ bool launch_nt(const DecodeArgs &a, cudaStream_t s)
 
 }  // namespace
 
-// The non-fused decode at head_dim 256 with the default block formats and up to
-// 24 rows per KV head.
+// The decode at head_dim 256 with the default block formats and up to 24 rows
+// per KV head.
 bool launch_decode_tmem(const DecodeArgs &a, cudaStream_t s)
 {
     const int rows = (a.n_q_heads / a.n_kv_heads) * a.T;

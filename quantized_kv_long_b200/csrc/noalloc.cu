@@ -13,8 +13,12 @@
 // The array is a file-scope __device__ object of KVQ_STATIC_SCRATCH_BYTES
 // (8 MiB): every GPU on which the library is loaded keeps those 8 MiB until
 // the process exits.  Host code never uses the array's name as an address:
-// the device address comes from cudaGetSymbolAddress, taken once per device
-// (with that device current) on the first call made on it.
+// the device address comes from cudaGetSymbolAddress, taken per device (with
+// that device current) on the first call made on it and kept in an atomic, so
+// that host threads calling at the same time may each look it up but never
+// race on the stored value.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace kvq {
@@ -32,8 +36,7 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_scratch[KVQ_STATIC_SCRATCH_BYTES];
 
-constexpr int MAX_DEVICES = 64;
-unsigned char *g_scratch_addr[MAX_DEVICES] = {};
+std::atomic<unsigned char *> g_scratch_addr[MAX_DEVICES];
 
 // Device address of this device's scratch array (looked up once per device).
 kvq_status scratch_address(unsigned char **out, const char *fn)
@@ -44,15 +47,17 @@ kvq_status scratch_address(unsigned char **out, const char *fn)
         return set_error(KVQ_ERR_CUDA, "%s: cudaGetDevice: %s", fn, cudaGetErrorString(e));
     if (dev < 0 || dev >= MAX_DEVICES)
         return set_error(KVQ_ERR_UNSUPPORTED, "%s: device %d beyond %d", fn, dev, MAX_DEVICES);
-    if (!g_scratch_addr[dev]) {
+    unsigned char *addr = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!addr) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_scratch);
         if (e != cudaSuccess || p == nullptr)
             return set_error(KVQ_ERR_CUDA, "%s: cudaGetSymbolAddress: %s", fn,
                              cudaGetErrorString(e));
-        g_scratch_addr[dev] = static_cast<unsigned char *>(p);
+        addr = static_cast<unsigned char *>(p);
+        g_scratch_addr[dev].store(addr, std::memory_order_release);
     }
-    *out = g_scratch_addr[dev];
+    *out = addr;
     return KVQ_OK;
 }
 
@@ -67,34 +72,35 @@ extern "C" kvq_status kvq_decode_merged_static(const kvq_layer *layers, int n_la
                                                float *lse, kvq_stream stream)
 {
     const char *fn = "kvq_decode_merged_static";
-    if (!layers || n_layers < 1 || n_layers > KVQ_MAX_LAYERS)
-        return set_error(KVQ_ERR_INVALID_ARG, "%s: bad layers / n_layers=%d", fn, n_layers);
-    if (chunk < 64 || chunk % 64 != 0)
-        return set_error(KVQ_ERR_INVALID_ARG, "%s: chunk=%d not a positive multiple of 64", fn,
-                         chunk);
-    const int D = layers[0].head_dim;
-    if (n_q_heads < 1 || T < 1 || D < 32 || n_kv < 1)
-        return set_error(KVQ_ERR_INVALID_ARG, "%s: bad shape", fn);
-    const int64_t rows = (int64_t)n_layers * T * n_q_heads;
-    const int64_t n_chunks = (n_kv + chunk - 1) / chunk;
-    // partials: out_part [rows][n_chunks][D] then lse_part [rows][n_chunks], 256-B aligned
-    const int64_t part_bytes = ((rows * n_chunks * D * 4 + 255) / 256) * 256;
-    const int64_t need = part_bytes + rows * n_chunks * 4;
-    if (need > (int64_t)KVQ_STATIC_SCRATCH_BYTES)
-        return set_error(KVQ_ERR_UNSUPPORTED,
-                         "%s: chunk partials need %lld bytes, more than the %lld-byte static "
-                         "scratch (fewer layers or larger chunks per call)",
-                         fn, (long long)need, (long long)KVQ_STATIC_SCRATCH_BYTES);
     unsigned char *base = nullptr;
     kvq_status st = scratch_address(&base, fn);
     if (st != KVQ_OK)
         return st;
-    float *out_part = reinterpret_cast<float *>(base);
-    float *lse_part = reinterpret_cast<float *>(base + part_bytes);
-    st = validate_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
-                         lse_part, fn);
+    // every argument is checked before any size is derived from it; the partial
+    // pointers given here are the array's start (the real lse_part offset follows)
+    st = validate_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale,
+                         reinterpret_cast<float *>(base), reinterpret_cast<float *>(base), fn);
     if (st != KVQ_OK)
         return st;
+    // validated: 1 <= n_layers <= KVQ_MAX_LAYERS, n_kv <= capacity, at most 2^30
+    // chunks and head_dim <= 512, so a row's partials take below 2^42 bytes and the
+    // row count test below keeps every product in range
+    const int D = layers[0].head_dim;
+    const int64_t rows = (int64_t)n_layers * T * n_q_heads;
+    const int64_t n_chunks = (n_kv + chunk - 1) / chunk;
+    const int64_t row_bytes = n_chunks * ((int64_t)D * 4 + 4);
+    // partials: out_part [rows][n_chunks][D] then lse_part [rows][n_chunks], 256-B aligned
+    const int64_t fits = rows <= (int64_t)KVQ_STATIC_SCRATCH_BYTES / row_bytes;
+    const int64_t part_bytes = fits ? ((rows * n_chunks * D * 4 + 255) / 256) * 256 : 0;
+    const int64_t need = fits ? part_bytes + rows * n_chunks * 4 : 0;
+    if (!fits || need > (int64_t)KVQ_STATIC_SCRATCH_BYTES)
+        return set_error(KVQ_ERR_UNSUPPORTED,
+                         "%s: %lld rows x %lld chunks of partials exceed the %lld-byte static "
+                         "scratch (fewer layers or larger chunks per call)",
+                         fn, (long long)rows, (long long)n_chunks,
+                         (long long)KVQ_STATIC_SCRATCH_BYTES);
+    float *out_part = reinterpret_cast<float *>(base);
+    float *lse_part = reinterpret_cast<float *>(base + part_bytes);
     st = validate_merge(out_part, lse_part, rows, (int)n_chunks, D, out, lse, fn);
     if (st != KVQ_OK)
         return st;

@@ -106,6 +106,7 @@ struct PfSmemHead {
     uint64_t raw_full[NR], raw_free[NR], k_full[NB_MAX], v_full[NB_MAX], s_full[NS], p_full[NS],
         pv_done[NS], q_ready;
     uint64_t mma_drain;              // one commit after the last MMA: all of them are done
+    uint64_t never;                  // test hook: a barrier that nothing completes
     uint64_t xch[N_SOFT];            // two softmax warps per quadrant: the final sums
     float xmx[2][2][BM];             // [warp half][phase parity][row]: tile max, then l
     uint32_t tmem_base;
@@ -286,6 +287,8 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
     const uint8_t *kg = a.layers.k[layer] + (int64_t)h * cap * KROW;
     const uint8_t *vg = a.layers.v[layer] + (int64_t)h * cap * VROW;
     volatile int *abort = &hd.abort;
+    // test hook: the first CTA's producer waits on a barrier that nothing completes
+    const bool hook_wait = a.test_timeout && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NR; ++i) {
@@ -303,6 +306,7 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         }
         ptx::mbar_init(&hd.q_ready, n_soft<PRE>());
         ptx::mbar_init(&hd.mma_drain, 1);
+        ptx::mbar_init(&hd.never, 1);
         for (int i = 0; i < N_SOFT; ++i)
             ptx::mbar_init(&hd.xch[i], 2);
         hd.abort = 0;
@@ -384,6 +388,42 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
 #pragma unroll
         for (int k = 0; k < NHALF; ++k)
             l[k] = 0.0f;
+        const int64_t row_out = ((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq;
+        uint32_t xph = 0;  // phases of the pair's exchange barrier used so far
+        // out = O / l and lse = (m + log2 l) ln 2 of this thread's row into dsto / dstl,
+        // once the PV of tile `last` is done; l = l[0] + l[1] (the two warps of a
+        // quadrant add their halves, half 0 first).  false: a wait ran out.
+        auto emit = [&](int last, float *dsto, float *dstl, uint32_t ph) -> bool {
+            bool done = wwait(&hd.pv_done[slot(last, NS)], par(last, NS));
+            float lt = l[0] + l[NHALF - 1];  // NH == 1: l of half 0 + l of half 1
+            if (NH == 2 && done) {
+                hd.xmx[hf][ph & 1][i] = l[0];
+                done = pair_sync(ph);
+                if (done)
+                    lt = hd.xmx[0][ph & 1][i] + hd.xmx[1][ph & 1][i];
+            }
+            if (!done)
+                return false;
+            ptx::tc_fence_after();
+            const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
+            float4 *op = reinterpret_cast<float4 *>(dsto);
+            for (int c = h0 * 8; c < h0 * 8 + 16 / NH; ++c) {
+                uint32_t r[16];
+                ptx::tmem_ld16(lane_addr + COL_O + 16 * c, r);
+                ptx::tmem_wait_ld();
+                if (live) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        op[c * 4 + v] = make_float4(__uint_as_float(r[4 * v]) * inv,
+                                                    __uint_as_float(r[4 * v + 1]) * inv,
+                                                    __uint_as_float(r[4 * v + 2]) * inv,
+                                                    __uint_as_float(r[4 * v + 3]) * inv);
+                }
+            }
+            if (live && h0 == 0)
+                *dstl = lt > 0.0f ? (m + log2f(lt)) * LN2 : -INFINITY;
+            return true;
+        };
         bool ok = true;
         for (int j = 0; ok && j < ntiles; ++j) {
             const int sb = slot(j, NS);
@@ -480,41 +520,9 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         if (!ok && lane == 0)
             fail();
         // ---- epilogue: out = O / l, lse = (m + log2 l) ln 2, l = l[0] + l[1]
-        if (ok && !*abort) {
-            const int last = ntiles - 1;
-            bool done = wwait(&hd.pv_done[slot(last, NS)], par(last, NS));
-            float lt = l[0] + l[NHALF - 1];  // NH == 1: l of half 0 + l of half 1
-            if (NH == 2 && done) {  // the pair adds its two halves, half 0 first
-                hd.xmx[hf][0][i] = l[0];
-                done = pair_sync(0);
-                if (done)
-                    lt = hd.xmx[0][0][i] + hd.xmx[1][0][i];
-            }
-            if (done) {
-                ptx::tc_fence_after();
-                const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-                float4 *op = reinterpret_cast<float4 *>(
-                    a.out + (((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq) * HD);
-                for (int c = h0 * 8; c < h0 * 8 + 16 / NH; ++c) {
-                    uint32_t r[16];
-                    ptx::tmem_ld16(lane_addr + COL_O + 16 * c, r);
-                    ptx::tmem_wait_ld();
-                    if (live) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            op[c * 4 + v] = make_float4(__uint_as_float(r[4 * v]) * inv,
-                                                        __uint_as_float(r[4 * v + 1]) * inv,
-                                                        __uint_as_float(r[4 * v + 2]) * inv,
-                                                        __uint_as_float(r[4 * v + 3]) * inv);
-                    }
-                }
-                if (live && h0 == 0)
-                    a.lse[((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq] =
-                        lt > 0.0f ? (m + log2f(lt)) * LN2 : -INFINITY;
-            } else if (lane == 0) {
-                fail();
-            }
-        }
+        if (ok && !*abort && !emit(ntiles - 1, a.out + row_out * HD, a.lse + row_out, xph++) &&
+            lane == 0)
+            fail();
     } else if (warp < W_PROD) {
         // ================================================================ dequant
         // Each of the 256 dequant threads owns one (key r, block bk) unit of every
@@ -569,6 +577,8 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         // The f16 tiles were expanded into the workspace: tile j of (layer, h) is one
         // 48 KB image of the three slots.  Slot kb is free once the QK^T (K^) and the
         // PV (V^) of tile j - NB are done; one transaction barrier covers the tile.
+        if (lane == 0 && hook_wait && !ptx::mbar_wait_bounded(&hd.never, 0, abort, WAIT_NS))
+            fail();
         if (lane == 0) {
             const int tiles_total = (int)((a.n_cached + a.T + BN - 1) / BN);
             const uint8_t *wsb = static_cast<const uint8_t *>(a.workspace) +
@@ -598,6 +608,8 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         }
     } else if (warp == W_PROD) {
         // ================================================================ copies
+        if (lane == 0 && hook_wait && !ptx::mbar_wait_bounded(&hd.never, 0, abort, WAIT_NS))
+            fail();
         if (lane == 0) {
             int issued = 0;
             for (int j = 0; j < ntiles; ++j) {
@@ -741,6 +753,19 @@ __global__ void __launch_bounds__(EXP_THREADS) prefill_expand_kernel(const Prefi
     const int64_t n_keys = a.n_cached + a.T;
     const int rows = (int)min((int64_t)BN, n_keys - (int64_t)t * BN);
     const int64_t cap = a.layers.cap[layer];
+    if (threadIdx.x == 0 && a.test_timeout && t == 0 && h == 0 && layer == 0) {
+        // test hook: a bounded wait on a barrier that nothing completes, before any copy
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+        int none = 0;
+        if (!ptx::mbar_wait_bounded(bar, 0, &none, WAIT_NS))
+            report_timeout(a.status);
+        ok_s = 0;
+    }
+    if (a.test_timeout && t == 0 && h == 0 && layer == 0) {
+        __syncthreads();
+        return;
+    }
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar, 1);
         ptx::fence_mbar_init();
@@ -812,7 +837,34 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
     }
     __syncthreads();
     const int64_t kend = a.n_cached + t0 + ntok;  // keys the last token sees
+    const bool PG = a.page_out != nullptr;  // per-page partials (see prefill_tc_kernel)
+    const int n_pages = (int)((a.n_cached + a.T + a.page - 1) / a.page);
+    // the partial of page pg of every row: out = acc / l, lse = m + ln l (0, -inf if
+    // the row saw nothing of it)
+    auto write_page = [&](int pg) {
+        for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
+            const int r = p / D, i = p % D;
+            const int t = t0 + r / G, g = r % G;
+            const int64_t row = ((int64_t)layer * a.T + t) * a.n_q_heads + h * G + g;
+            const float l = l_s[r];
+            a.page_out[(row * n_pages + pg) * D + i] = (l > 0.0f) ? acc[p] / l : 0.0f;
+            if (i == 0)
+                a.page_lse[row * n_pages + pg] = (l > 0.0f) ? m_s[r] + logf(l) : -INFINITY;
+        }
+    };
     for (int64_t j0 = 0; j0 < kend; j0 += EX_TILE) {
+        if (PG && j0 > 0 && j0 % a.page == 0) {
+            // page boundary: write the previous page, restart the (max, sum, acc)
+            write_page((int)(j0 / a.page) - 1);
+            __syncthreads();
+            for (int p = threadIdx.x; p < R * D; p += blockDim.x)
+                acc[p] = 0.0f;
+            for (int r = threadIdx.x; r < R; r += blockDim.x) {
+                m_s[r] = -INFINITY;
+                l_s[r] = 0.0f;
+            }
+            __syncthreads();
+        }
         for (int p = threadIdx.x; p < R * EX_TILE; p += blockDim.x) {
             const int r = p / EX_TILE, jj = p % EX_TILE;
             const int64_t j = j0 + jj;
@@ -876,6 +928,21 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
         }
         __syncthreads();
     }
+    if (PG) {
+        const int pl = (int)((kend - 1) / a.page);  // the page of the last key read
+        write_page(pl);
+        // pages past the keys of this block: nothing visible
+        for (int pg = pl + 1; pg < n_pages; ++pg)
+            for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
+                const int r = p / D, i = p % D;
+                const int t = t0 + r / G, g = r % G;
+                const int64_t row = ((int64_t)layer * a.T + t) * a.n_q_heads + h * G + g;
+                a.page_out[(row * n_pages + pg) * D + i] = 0.0f;
+                if (i == 0)
+                    a.page_lse[row * n_pages + pg] = -INFINITY;
+            }
+        return;
+    }
     for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
         const int r = p / D, i = p % D;
         const int t = t0 + r / G, g = r % G;
@@ -907,47 +974,35 @@ bool prefill_supported(int n_q_heads, int n_kv_heads, int head_dim)
 void launch_prefill(const PrefillArgs &a, cudaStream_t s)
 {
     const int G = a.n_q_heads / a.n_kv_heads;
-    // tokens whose rows see fewer than PF_MIN_KEYS keys take the exact kernel
-    // (host test hook KVQ_PREFILL_TC_MIN_KEYS moves the threshold)
-    int64_t min_keys = PF_MIN_KEYS;
-    if (const char *e = getenv("KVQ_PREFILL_TC_MIN_KEYS"))
-        min_keys = atoll(e);
-    int64_t t_split = min_keys - 1 - a.n_cached;
+    // tokens whose rows see fewer than PF_MIN_KEYS keys take the exact kernel; so do
+    // all rows when per-page partials are asked for (a page is a short context, where
+    // the tensor-core path's f16 rounding of V^ and P is not within the tolerance)
+    int64_t t_split = PF_MIN_KEYS - 1 - a.n_cached;
     t_split = t_split < 0 ? 0 : (t_split > a.T ? a.T : t_split);
+    if (a.page_out)
+        t_split = a.T;
     if (a.head_dim != HD)
         t_split = a.T;  // the tensor-core path is built for head_dim 256
     if (t_split > 0) {
         const int tb = max(1, 32 / G);
         const size_t smem = sizeof(float) * ((size_t)2 * tb * G * a.head_dim +
                                              (size_t)tb * G * EX_TILE + 3 * (size_t)tb * G);
-        static bool attr_ex[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (smem > 48 * 1024 && dev >= 0 && dev < 64 && !attr_ex[dev]) {
-            cudaFuncSetAttribute(prefill_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-            attr_ex[dev] = true;
-        }
+        static std::atomic<int> smem_ex[MAX_DEVICES];
+        ensure_smem(reinterpret_cast<const void *>(prefill_exact_kernel), smem_ex, (int)smem);
         dim3 grid((unsigned)((t_split + tb - 1) / tb), a.n_kv_heads, a.n_layers);
         prefill_exact_kernel<<<grid, EX_THREADS, smem, s>>>(a, tb, (int)t_split);
     }
     if (t_split < a.T) {
         // with a workspace (the caller checked its size), expand the f16 tiles once
         const bool pre = a.workspace != nullptr;
-        static bool attr_tc[2][64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev >= 0 && dev < 64 && !attr_tc[pre][dev]) {
-            if (pre) {
-                cudaFuncSetAttribute(prefill_tc_kernel<true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, pf_smem<true>());
-                cudaFuncSetAttribute(prefill_expand_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, EXP_SMEM);
-            } else {
-                cudaFuncSetAttribute(prefill_tc_kernel<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, pf_smem<false>());
-            }
-            attr_tc[pre][dev] = true;
+        static std::atomic<int> smem_tc[2][MAX_DEVICES], smem_exp[MAX_DEVICES];
+        if (pre) {
+            ensure_smem(reinterpret_cast<const void *>(prefill_tc_kernel<true>), smem_tc[1],
+                        pf_smem<true>());
+            ensure_smem(reinterpret_cast<const void *>(prefill_expand_kernel), smem_exp, EXP_SMEM);
+        } else {
+            ensure_smem(reinterpret_cast<const void *>(prefill_tc_kernel<false>), smem_tc[0],
+                        pf_smem<false>());
         }
         const int row0 = (int)t_split * G;
         const int rows = a.T * G - row0;

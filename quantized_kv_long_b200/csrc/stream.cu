@@ -80,8 +80,7 @@ int placement(const void *p)
 
 int fail_copy_layer()
 {
-    const char *e = getenv("KVQ_TEST_FAIL_COPY_LAYER");
-    return e ? atoi(e) : -1;
+    return test_hooks().stream_fail_layer.load(std::memory_order_relaxed);
 }
 
 }  // namespace

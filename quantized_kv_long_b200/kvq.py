@@ -58,6 +58,11 @@ class kvq_layer(ctypes.Structure):
                 ("k_type", ctypes.c_int32), ("v_type", ctypes.c_int32)]
 
 
+class kvq_test_hooks(ctypes.Structure):
+    _fields_ = [("decode_general", ctypes.c_int32), ("decode_timeout", ctypes.c_int32),
+                ("prefill_timeout", ctypes.c_int32), ("stream_fail_layer", ctypes.c_int32)]
+
+
 class KvqError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{message} [{status}: {kvq_status_string(status)}]")
@@ -88,6 +93,7 @@ _SIGS = {
     "kvq_status_string": ([_I32], ctypes.c_char_p),
     "kvq_last_error": ([], ctypes.c_char_p),
     "kvq_version": ([], _I32),
+    "kvq_test_set_hooks": ([ctypes.POINTER(kvq_test_hooks)], _I32),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -170,12 +176,11 @@ def kvq_merge_lse(out_part, lse_part, rows: int, n_chunks: int, head_dim: int, o
 
 
 def kvq_decode_step(layers, k_new, v_new, q, n_q_heads: int, T: int, n_kv: int, chunk: int,
-                    scale: float, out_part, lse_part, out, lse, workspace, ws_bytes: int | None = None,
+                    scale: float, out_part, lse_part, out, lse, workspace=None, ws_bytes: int = 0,
                     stream=None) -> None:
-    """Append + decode + merge in one launch (see include/kvq.h)."""
+    """Append + decode + merge as three launches on ``stream`` (see include/kvq.h);
+    ``workspace`` is reserved and not read."""
     arr, n = _layers(layers)
-    if ws_bytes is None:
-        ws_bytes = workspace.numel() * workspace.element_size()
     _check(_lib.kvq_decode_step(arr, n, _ptr(k_new), _ptr(v_new), _ptr(q), n_q_heads, T, n_kv,
                                 chunk, scale, _ptr(out_part), _ptr(lse_part), _ptr(out), _ptr(lse),
                                 _ptr(workspace), ws_bytes, _stream(stream)))
@@ -230,6 +235,29 @@ def kvq_prefill_workspace_bytes(n_layers: int, n_kv_heads: int, head_dim: int,
 def kvq_workspace_bytes(op: int, n_layers: int, n_q_heads: int, n_kv_heads: int, T: int,
                         head_dim: int) -> int:
     return _lib.kvq_workspace_bytes(op, n_layers, n_q_heads, n_kv_heads, T, head_dim)
+
+
+def kvq_test_set_hooks(decode_general: bool = False, decode_timeout: bool = False,
+                       prefill_timeout: bool = False, stream_fail_layer: int = -1) -> None:
+    """Set the library's process-wide test hooks (all off by default)."""
+    h = kvq_test_hooks(int(decode_general), int(decode_timeout), int(prefill_timeout),
+                       stream_fail_layer)
+    _check(_lib.kvq_test_set_hooks(ctypes.byref(h)))
+
+
+class test_hooks:
+    """Context manager: the given test hooks on inside the block, all off after it."""
+
+    def __init__(self, **kw):
+        self.kw = kw
+
+    def __enter__(self):
+        kvq_test_set_hooks(**self.kw)
+        return self
+
+    def __exit__(self, *exc):
+        _check(_lib.kvq_test_set_hooks(None))
+        return False
 
 
 def kvq_check(stream=None) -> None:

@@ -118,12 +118,12 @@ def test_merge_validation(kvq):
 
 
 def test_decode_step_validation(kvq):
-    """kvq_decode_step: the decode and merge checks plus k_new / v_new and the workspace
-    (16 layers x 4 KV heads x 4 bytes = 256 bytes here)."""
+    """kvq_decode_step: the decode and merge checks plus k_new / v_new, all before the
+    first launch; the workspace is reserved (0 bytes, not read)."""
     L = [_layer(kvq)] * 16
-    assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE_STEP, 16, 24, 4, 4, 256) == 256
+    assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE_STEP, 16, 24, 4, 4, 256) == 0
     ok = dict(k_new=A, v_new=A, q=A, n_q_heads=24, T=4, n_kv=1024, chunk=256, scale=1 / 16,
-              out_part=A, lse_part=A, out=A, lse=A, workspace=A, ws_bytes=256, stream=0)
+              out_part=A, lse_part=A, out=A, lse=A, workspace=None, ws_bytes=0, stream=0)
 
     def call(**kw):
         d = dict(ok)
@@ -141,9 +141,6 @@ def test_decode_step_validation(kvq):
     bad(kvq.KVQ_ERR_INVALID_ARG, n_kv=1025)
     bad(kvq.KVQ_ERR_ALIGNMENT, out=A + 4)
     bad(kvq.KVQ_ERR_INVALID_ARG, lse=None)
-    bad(kvq.KVQ_ERR_WORKSPACE, workspace=None)
-    bad(kvq.KVQ_ERR_WORKSPACE, ws_bytes=252)
-    bad(kvq.KVQ_ERR_WORKSPACE, workspace=A + 2)
 
 
 def test_prefill_validation(kvq):
@@ -159,7 +156,8 @@ def test_prefill_validation(kvq):
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, page=100)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, n_cached=4000)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, page_out=A)
-    _raises(kvq, kvq.KVQ_ERR_UNSUPPORTED, call, page_out=A, page_lse=A)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, call, page_out=A + 4, page_lse=A)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, call, page_out=A, page_lse=A + 2)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, call, T=0)
     _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, call, out=A + 4)
 
@@ -174,7 +172,20 @@ def test_stream_validation(kvq):
 
 def test_workspace_query(kvq):
     assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE, 16, 24, 4, 4, 256) == 0
+    # prefill requires no workspace; its optional one is kvq_prefill_workspace_bytes
+    assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_PREFILL, 16, 24, 4, 2048, 256) == 0
+    assert kvq.kvq_prefill_workspace_bytes(16, 4, 256, 264192) > 0
+    assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE_STEP, 16, 24, 4, 4, 256) == 0
     assert kvq.kvq_workspace_bytes(99, 1, 1, 1, 1, 32) == ctypes.c_size_t(-1).value
+
+
+def test_test_hooks_set_and_clear(kvq):
+    """The hooks are plain process-wide switches: set, then cleared by the context
+    manager (host only; no kernel runs)."""
+    with kvq.test_hooks(decode_general=True, stream_fail_layer=3):
+        pass
+    kvq.kvq_test_set_hooks()  # all off
+    assert kvq._lib.kvq_test_set_hooks(None) == kvq.KVQ_OK
 
 
 def test_resident_layers_plan(kvq):

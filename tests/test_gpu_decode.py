@@ -24,13 +24,10 @@ def kvq():
 
 
 @pytest.fixture(params=["tc", "simple"])
-def kernel(request, monkeypatch):
+def kernel(request, kvq):
     """Run a case on the tiled tensor-core kernel and on the general kernel."""
-    if request.param == "simple":
-        monkeypatch.setenv("KVQ_DECODE_KERNEL", "simple")
-    else:
-        monkeypatch.delenv("KVQ_DECODE_KERNEL", raising=False)
-    return request.param
+    with kvq.test_hooks(decode_general=request.param == "simple"):
+        yield request.param
 
 
 def run_decode(kvq, cache, q, Hq, T, n_kv, chunk, scale, layers=None):
@@ -144,24 +141,23 @@ def test_tc_stage_edges(kvq, n_kv, chunk):
 
 
 @pytest.mark.parametrize("T", [1, 4])
-def test_bounded_wait_times_out_and_context_survives(kvq, monkeypatch, T):
+def test_bounded_wait_times_out_and_context_survives(kvq, T):
     """A wait on a barrier that nothing completes runs out after about a
     second: the kernel ends, kvq_check reports KVQ_ERR_TIMEOUT once, and the
-    next call on the same context is correct again.  T = 1 runs the pair
-    kernel, T = 4 the role-split kernel."""
+    next call on the same context is correct again (the persistent kernel, one
+    and three n-tiles of rows)."""
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=512)
     cache, orc = fill_both(w, [0], 512, 512)
     q = q_all(w, [0], T)
-    monkeypatch.setenv("KVQ_TEST_DECODE_TIMEOUT", "1")
     qt = torch.from_numpy(q).cuda()
     op = torch.empty((1, T, 24, 1, 256), device="cuda")
     lp = torch.empty((1, T, 24, 1), device="cuda")
-    kvq.kvq_decode_attn(cache.layers(), qt, 24, T, 512, 512, w.scale, op, lp)
-    with pytest.raises(kvq.KvqError) as e:
-        kvq.kvq_check()
+    with kvq.test_hooks(decode_timeout=True):
+        kvq.kvq_decode_attn(cache.layers(), qt, 24, T, 512, 512, w.scale, op, lp)
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_check()
     assert e.value.status == kvq.KVQ_ERR_TIMEOUT
     kvq.kvq_check()  # the status word was cleared
-    monkeypatch.delenv("KVQ_TEST_DECODE_TIMEOUT")
     op2, lp2, out, lse = run_decode(kvq, cache, q, 24, T, 512, 512, w.scale)
     rp, rl = oracle.decode_attn(orc[0][0], orc[0][1], q[0], 512, 512, w.scale)
     assert_attn_close(op2[0], lp2[0], rp, rl, "after timeout")

@@ -69,15 +69,14 @@ def test_decode_step_three_launches(kvq, k_type, v_type):
     v_new = torch.from_numpy(wl.kv_rows(w, 0, 1, n0, n_kv)[None]).cuda()
     q = torch.from_numpy(q_all(w, [0], T)).cuda()
     outs = []
-    for fused, c in ((False, ca), (True, cb)):
+    for one_call, c in ((False, ca), (True, cb)):
         op = torch.full((1, T, Hq, C, D), float("nan"), device="cuda")
         lp = torch.full((1, T, Hq, C), float("nan"), device="cuda")
         out = torch.full((1, T, Hq, D), float("nan"), device="cuda")
         lse = torch.full((1, T, Hq), float("nan"), device="cuda")
-        if fused:
-            ws = torch.zeros(H, dtype=torch.int32, device="cuda")
+        if one_call:
             kvq.kvq_decode_step(c, k_new, v_new, q, Hq, T, n_kv, chunk, w.scale, op, lp, out,
-                                lse, ws)
+                                lse)
         else:
             kvq.kvq_append(c, k_new, v_new, n0, T)
             kvq.kvq_decode_attn(c, q, Hq, T, n_kv, chunk, w.scale, op, lp)

@@ -112,3 +112,54 @@ def test_prefill262k_full_size_sampled(kvq):
                                   w.scale)
         assert_attn_close(out[l, ts, hs].cpu().numpy(), lse[l, ts, hs].cpu().numpy(), ro, rl,
                           f"prefill262k layer {l}")
+
+
+@pytest.mark.parametrize("Hq,H,n_cached,T,page", [
+    (6, 1, 16300, 300, 256),    # exact + tensor-core rows; later pages fully masked for early rows
+    (6, 1, 16384, 512, 256),    # tensor-core CTAs whose keys end before the last page
+    (24, 4, 16448, 128, 4096),  # the default heads, five pages
+])
+def test_page_partials(kvq, Hq, H, n_cached, T, page):
+    """The optional per-page partials [T][Hq][n_pages][D] and lse, element by element
+    against the oracle's pages (a page a row sees nothing of is out = 0, lse = -inf),
+    and out / lse as their merge against the oracle's one-pass result."""
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=n_cached, T=T, n_q_heads=Hq, n_kv_heads=H)
+    n = n_cached + T
+    cache, orc = fill_both(w, [0], n, -(-n // 8) * 8)
+    q = np.stack([wl.q_rows(w, 0, T)])
+    D, n_pages = w.head_dim, -(-n // page)
+    out = torch.full((1, T, Hq, D), float("nan"), device="cuda")
+    lse = torch.full((1, T, Hq), float("nan"), device="cuda")
+    po = torch.full((1, T, Hq, n_pages, D), float("nan"), device="cuda")
+    pl = torch.full((1, T, Hq, n_pages), float("nan"), device="cuda")
+    kvq.kvq_prefill_attn(cache.layers(), torch.from_numpy(q).cuda(), Hq, T, n_cached, page,
+                         w.scale, out, lse, page_out=po, page_lse=pl)
+    kvq.kvq_check()
+    ro, rl, rpo, rpl = oracle.prefill_attn(orc[0][0], orc[0][1], q[0], n_cached, page, w.scale,
+                                           pages=True)
+    gpo, gpl = po.cpu().numpy()[0], pl.cpu().numpy()[0]
+    assert_attn_close(gpo, gpl, rpo, rpl, "page partials")
+    masked = np.isneginf(rpl)
+    assert np.isneginf(gpl[masked]).all() and (gpo[masked] == 0).all()
+    assert_attn_close(out.cpu().numpy()[0], lse.cpu().numpy()[0], ro, rl, "merged pages")
+
+
+@pytest.mark.parametrize("expand", [False, True])
+def test_prefill_bounded_wait_times_out_and_context_survives(kvq, expand):
+    """The prefill test hook makes one bounded wait of the first CTA of each
+    tensor-core launch (the tile expansion and the attention kernel) run out after
+    about a second: kvq_check reports KVQ_ERR_TIMEOUT, the CTAs free their tensor
+    memory, and the next call on the same context matches the oracle."""
+    n_cached, T = 16448, 128
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=n_cached, T=T)
+    n = n_cached + T
+    cache, orc = fill_both(w, [0], n, -(-n // 8) * 8)
+    q = np.stack([wl.q_rows(w, 0, T)])
+    with kvq.test_hooks(prefill_timeout=True):
+        with pytest.raises(kvq.KvqError) as e:
+            run_prefill(kvq, cache, q, w.n_q_heads, T, n_cached, w.scale, expand=expand)
+    assert e.value.status == kvq.KVQ_ERR_TIMEOUT
+    kvq.kvq_check()  # cleared
+    out, lse = run_prefill(kvq, cache, q, w.n_q_heads, T, n_cached, w.scale, expand=expand)
+    ro, rl = oracle.prefill_attn(orc[0][0], orc[0][1], q[0], n_cached, 1024, w.scale)
+    assert_attn_close(out[0], lse[0], ro, rl, "after timeout")

@@ -1,12 +1,9 @@
-"""kvq_decode_step (append + decode + merge in one launch) on the GPU.
+"""kvq_decode_step (append, decode and merge issued by one call) on the GPU.
 
-The fused step must give exactly what the three separate calls give: the
-same cache bytes (the in-kernel append uses the append kernel's arithmetic),
-the same chunk partials (the same decode kernel body), and the same merged
-rows (the last CTA of each KV head runs the merge kernel's per-row routine,
-whose order of operations is fixed).  So the comparison is bit-for-bit, on
-cases that put the new rows in one chunk, across a chunk boundary, and make
-up the whole cache; one case is also checked against the oracle.
+The step must give exactly what the three separate calls give: the same
+cache bytes, the same chunk partials and the same merged rows, bit for bit,
+on cases that put the new rows in one chunk, across a chunk boundary, and
+make up the whole cache; one case is also checked against the oracle.
 """
 import numpy as np
 import pytest
@@ -47,7 +44,7 @@ def _outputs(L, T, Hq, C, D):
 
 
 def run_both(kvq, w, n_layers, T, n_kv, chunk):
-    """The three-call step on one cache and the fused step on an identical one."""
+    """The three-call step on one cache and kvq_decode_step on an identical one."""
     cap = -(-n_kv // 8) * 8
     n0 = n_kv - T
     Hq, H, D = w.n_q_heads, w.n_kv_heads, w.head_dim
@@ -62,13 +59,11 @@ def run_both(kvq, w, n_layers, T, n_kv, chunk):
     kvq.kvq_append(ca, k_new, v_new, n0, T)
     kvq.kvq_decode_attn(ca, q, Hq, T, n_kv, chunk, w.scale, op_a, lp_a)
     kvq.kvq_merge_lse(op_a, lp_a, n_layers * T * Hq, C, D, out_a, lse_a)
-    # one launch; the workspace starts as garbage (the call clears it)
+    # one call (no workspace)
     op_b, lp_b, out_b, lse_b = _outputs(n_layers, T, Hq, C, D)
-    ws_bytes = kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE_STEP, n_layers, Hq, H, T, D)
-    assert ws_bytes == n_layers * H * 4
-    ws = torch.full((ws_bytes // 4,), 12345, dtype=torch.int32, device="cuda")
+    assert kvq.kvq_workspace_bytes(kvq.KVQ_OP_DECODE_STEP, n_layers, Hq, H, T, D) == 0
     kvq.kvq_decode_step(cb, k_new, v_new, q, Hq, T, n_kv, chunk, w.scale, op_b, lp_b, out_b,
-                        lse_b, ws)
+                        lse_b)
     kvq.kvq_check()
     for l in range(n_layers):
         assert torch.equal(ca.k[l], cb.k[l]), f"K cache bytes, layer {l}"
@@ -102,7 +97,7 @@ def test_step_all_rows_new(kvq):
 
 
 def test_step_many_chunks_against_oracle(kvq):
-    """chunk 64: 157 partials per row merged in-kernel; checked against the oracle too."""
+    """chunk 64: 157 partials per row; checked against the oracle too."""
     n_kv, T, chunk = 10000, 4, 64
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=n_kv)
     cache, q, out, lse = run_both(kvq, w, 1, T, n_kv, chunk)
@@ -110,11 +105,11 @@ def test_step_many_chunks_against_oracle(kvq):
     oracle.append(kc, vc, wl.kv_rows(w, 0, 0, 0, n_kv), wl.kv_rows(w, 0, 1, 0, n_kv), 0)
     rp, rl = oracle.decode_attn(kc, vc, q[0], n_kv, chunk, w.scale)
     ro, rlse = oracle.merge_lse(rp, rl)
-    assert_attn_close(out[0], lse[0], ro, rlse, "fused step vs oracle")
+    assert_attn_close(out[0], lse[0], ro, rlse, "decode step vs oracle")
 
 
-def test_step_general_kernel_path(kvq, monkeypatch):
-    """Shapes outside the tiled kernel (forced here) run as three launches, same results."""
-    monkeypatch.setenv("KVQ_DECODE_KERNEL", "simple")
+def test_step_general_kernel_path(kvq):
+    """The general decode kernel (forced here): the same bit-identity."""
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=3001)
-    run_both(kvq, w, 1, 4, 3001, 512)
+    with kvq.test_hooks(decode_general=True):
+        run_both(kvq, w, 1, 4, 3001, 512)

@@ -76,24 +76,22 @@ def test_streamed_equals_resident_and_oracle(kvq, T):
         assert_attn_close(so[l], sl[l], mo, ml, f"streamed layer {l}")
 
 
-def test_injected_copy_failure(kvq, monkeypatch):
+def test_injected_copy_failure(kvq):
     n_kv, chunk = 5000, 1024
     w, dev, orc, host, slots, q = _setup(kvq, n_layers=4)
-    monkeypatch.setenv("KVQ_TEST_FAIL_COPY_LAYER", "2")
     Hq, D = w.n_q_heads, w.head_dim
     C = -(-n_kv // chunk)
     op = torch.empty((1, Hq, C, D), device="cuda")
     lp = torch.empty((1, Hq, C), device="cuda")
     out = torch.full((4, 1, Hq, D), float("nan"), device="cuda")
     lse = torch.full((4, 1, Hq), float("nan"), device="cuda")
-    with pytest.raises(kvq.KvqError) as e:
+    with kvq.test_hooks(stream_fail_layer=2), pytest.raises(kvq.KvqError) as e:
         kvq.kvq_stream_decode(host, slots, q, Hq, 1, n_kv, chunk, w.scale, op, lp, out, lse,
                               compute=torch.cuda.current_stream(), copy=torch.cuda.Stream())
     assert e.value.status == kvq.KVQ_ERR_COPY
     kvq.kvq_check()  # the work already enqueued completes; the context stays usable
     o = out.cpu().numpy()
     assert np.isfinite(o[:2]).all() and np.isnan(o[2:]).all()
-    monkeypatch.delenv("KVQ_TEST_FAIL_COPY_LAYER")
     so, sl = _streamed(kvq, w, host, slots, q, n_kv, chunk, 1)
     assert np.isfinite(so).all()
 
