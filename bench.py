@@ -496,7 +496,22 @@ def run_prefill(args, w: wl.Workload) -> dict | None:
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     # the f16 key tiles expanded once per call (the timed region includes the expansion)
-    ws_bytes = 0 if args.no_expand else kvq.kvq_prefill_workspace_bytes(L, w.n_kv_heads, D, nc + T)
+    # into a workspace of whole slabs (one slab per (layer, KV head) pair) within
+    # --ws-mib; 0 = a slab for every pair
+    full = kvq.kvq_prefill_workspace_bytes(L, w.n_kv_heads, D, nc + T)
+    slab = kvq.kvq_prefill_workspace_bytes(1, 1, D, nc + T)
+    ws_bytes = full if args.ws_mib == 0 else min(full, (args.ws_mib << 20) // slab * slab)
+    if args.no_expand:
+        ws_bytes = 0
+    elif ws_bytes < slab:
+        raise SystemExit(f"--ws-mib {args.ws_mib} holds no slab of {slab} bytes")
+    n_pairs = L * w.n_kv_heads
+    slabs = ws_bytes // slab if ws_bytes else 0
+    if 2 <= slabs < n_pairs:  # chunks alternate between two halves: an odd slab is unused
+        slabs -= slabs % 2
+        ws_bytes = slabs * slab
+    chunk = n_pairs if slabs >= n_pairs else max(1, slabs // 2)
+    n_chunks = -(-n_pairs // chunk) if ws_bytes else 0
     ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=device) if ws_bytes else None
 
     def step(i=None):
@@ -540,19 +555,21 @@ def run_prefill(args, w: wl.Workload) -> dict | None:
             "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": w.n_kv_heads,
                        "head_dim": D, "cached": nc, "new_tokens": T, "seed": w.seed,
                        "flop_per_step": fl, "workspace_bytes": ws_bytes,
-                       "key_tiles": ("expanded once per call into the workspace" if ws_bytes
-                                     else "dequantized in each CTA")},
+                       "key_tiles": (f"expanded once per call into {slabs} workspace slabs, "
+                                     f"{n_chunks} chunk(s) of {chunk} (layer, KV head) pairs"
+                                     if ws_bytes else "dequantized in each CTA")},
             "query_tok_per_s": round(world * T / (ms * 1e-3), 1),
             "layer_query_tok_per_s": round(world * L * T / (ms * 1e-3), 1),
             "roofline": {"bound": "tensor",
-                         "kernel": ("kvq_prefill_attn (16 layers): tile expansion + prefill, 2 "
-                                    "launches" if ws_bytes else "kvq_prefill_attn (16 layers, 1 launch)"),
+                         "kernel": (f"kvq_prefill_attn ({L} layers): tile expansion + prefill, "
+                                    f"{2 * n_chunks} launches" if ws_bytes else
+                                    f"kvq_prefill_attn ({L} layers, 1 launch)"),
                          "achieved": round(fl / (k_ms * 1e-3) / 1e12, 2), "peak": peak,
                          "peak_kind": kind, "unit": "TFLOP/s",
                          "frac": round(fl / (k_ms * 1e-3) / 1e12 / peak, 4),
                          "traffic": tr["dram_bytes_per_layer"] * L if tr else None,
                          "launch_ms": round(k_ms, 3)},
-            "gpu_launches": (3 if ws_bytes else 2) * args.steps,
+            "gpu_launches": (1 + (2 * n_chunks if ws_bytes else 1)) * args.steps,
             "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
                        "reasons": cl["reasons"], "samples": cl["samples"]},
         }
@@ -644,6 +661,9 @@ def main(argv=None) -> int:
     ap.add_argument("--config", default="verify262k",
                     choices=["verify262k", "decode65k", "tiny", "prefill262k", "stream262k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ws-mib", type=int, default=2048,
+                    help="prefill262k: workspace for the expanded key tiles, MiB (whole slabs "
+                         "of one (layer, KV head) each; 0 = one slab per pair, 26 GB)")
     ap.add_argument("--no-expand", action="store_true",
                     help="prefill262k: no workspace; every CTA dequantizes its key tiles")
     ap.add_argument("--budget-mib", type=int, default=None,

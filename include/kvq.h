@@ -267,17 +267,26 @@ kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k
  *            by this call after the prefill kernels).
  *  workspace optional, device, 256-B aligned.  NULL: each CTA of the
  *            tensor-core path dequantizes the key tiles it reads.  Otherwise
- *            ws_bytes >= kvq_prefill_workspace_bytes(n_layers, n_kv_heads,
- *            head_dim, n_cached + T) and the call first expands every key tile
- *            once into the workspace (f16 K^hi, K^lo, V^: 1,536 B per key and KV
- *            head at head_dim 256), which the tensor-core kernel then copies in
- *            without dequantizing (every row tile of a KV head reads the same
- *            keys).  Same results bit for bit.  Ignored when the tensor-core
- *            path does not run.  Owned by the caller; not used after the call's
+ *            the call expands the key tiles of each (layer, KV head) pair once
+ *            into a "slab" of the workspace (f16 K^hi, K^lo, V^: 1,536 B per
+ *            key at head_dim 256; one slab = kvq_prefill_workspace_bytes(1, 1,
+ *            head_dim, n_cached + T)), which the tensor-core kernel then copies
+ *            in without dequantizing (every row tile of a pair reads the same
+ *            keys).  ws_bytes must hold at least one slab.  With a slab for
+ *            every pair (kvq_prefill_workspace_bytes(n_layers, n_kv_heads,
+ *            head_dim, n_cached + T)) one expansion and one attention launch
+ *            cover the call; with fewer, the pairs go in chunks of
+ *            floor(slabs / 2) through the two halves of the workspace,
+ *            alternating between `stream` and a second stream of the library
+ *            (forked from and joined back into `stream` with events, so the
+ *            call stays stream-ordered and can be captured in a CUDA graph);
+ *            with one slab, one pair at a time on `stream`.  All sizes give
+ *            the same results bit for bit.  Ignored when the tensor-core path
+ *            does not run.  Owned by the caller; not used after the call's
  *            work completes.
  * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (group size > 32, block formats
- *         other than Q8_0 K / Q4_0 V), WORKSPACE (a workspace smaller than
- *         needed), CUDA. */
+ *         other than Q8_0 K / Q4_0 V), WORKSPACE (a workspace smaller than one
+ *         slab), CUDA. */
 kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
                             int n_q_heads, int T, int64_t n_cached, int page, float scale,
                             float *out, float *lse, float *page_out, float *page_lse,
@@ -371,9 +380,11 @@ kvq_status kvq_decode_merged_static(const kvq_layer *layers, int n_layers, const
 /* Housekeeping                                                            */
 /* ---------------------------------------------------------------------- */
 
-/* Bytes of the optional kvq_prefill_attn workspace for n_keys = n_cached + T
- * keys: n_layers * n_kv_heads * ceil(n_keys / 32) * 49,152 at head_dim 256;
- * 0 when the shape has no tensor-core path (head_dim != 256). */
+/* Bytes of the optional kvq_prefill_attn workspace that holds a slab for every
+ * (layer, KV head) pair, for n_keys = n_cached + T keys: n_layers * n_kv_heads *
+ * ceil(n_keys / 32) * 49,152 at head_dim 256 (n_layers = n_kv_heads = 1 gives
+ * one slab, the smallest usable workspace); 0 when the shape has no
+ * tensor-core path (head_dim != 256). */
 size_t kvq_prefill_workspace_bytes(int n_layers, int n_kv_heads, int head_dim, int64_t n_keys);
 
 #define KVQ_OP_DECODE 1

@@ -398,13 +398,13 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
     // optional workspace: the f16 key tiles of the tensor-core path, expanded once
     a.workspace = nullptr;
     a.ws_bytes = 0;
-    const size_t exp = prefill_expand_bytes(n_layers, H, D, n_cached + T);
-    if (workspace != nullptr && exp > 0) {
-        if (ws_bytes < exp)
+    const size_t slab = prefill_slab_bytes(D, n_cached + T);
+    if (workspace != nullptr && slab > 0) {
+        if (ws_bytes < slab)
             return set_error(KVQ_ERR_WORKSPACE,
-                             "%s: workspace of %zu bytes given, the expanded tiles need %zu "
-                             "(kvq_prefill_workspace_bytes); pass NULL to dequantize in place",
-                             fn, ws_bytes, exp);
+                             "%s: workspace of %zu bytes given, one (layer, KV head) of expanded "
+                             "key tiles needs %zu; pass NULL to dequantize in place",
+                             fn, ws_bytes, slab);
         if (!aligned(workspace, 256))
             return set_error(KVQ_ERR_ALIGNMENT, "%s: workspace not 256-byte aligned", fn);
         a.workspace = workspace;
@@ -412,7 +412,9 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
     }
     KVQ_TRY(status_word(&a.status));
     a.test_timeout = test_hooks().prefill_timeout.load(std::memory_order_relaxed);
-    launch_prefill(a, as_stream(stream));
+    if (!launch_prefill(a, as_stream(stream)))
+        return set_error(KVQ_ERR_CUDA, "%s: setting up the second stream of the chunked "
+                         "expansion failed", fn);
     KVQ_TRY(check_launch(fn));
     if (page_out) {
         // the kernels wrote the per-page partials; out and lse are their merge

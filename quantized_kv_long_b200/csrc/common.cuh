@@ -126,12 +126,16 @@ struct PrefillArgs {
     size_t ws_bytes;
     unsigned int *status;
     int test_timeout;  // test hook: one bounded wait of each tensor-core launch runs out
+    int pair0;         // first (layer, KV head) pair, layer * n_kv_heads + head, of a launch
 };
 size_t prefill_workspace_bytes(int n_layers, int n_q_heads, int n_kv_heads, int T, int head_dim);
 // Optional workspace of the tensor-core path: the f16 key tiles expanded once per
 // call (0 if the shape has no such path).  n_keys = n_cached + T.
 size_t prefill_expand_bytes(int n_layers, int n_kv_heads, int head_dim, int64_t n_keys);
+// One (layer, KV head) pair's expanded key tiles: the smallest usable workspace.
+size_t prefill_slab_bytes(int head_dim, int64_t n_keys);
 bool prefill_supported(int n_q_heads, int n_kv_heads, int head_dim);
-void launch_prefill(const PrefillArgs &a, cudaStream_t s);
+// false: a stream or event for the chunked expansion could not be set up.
+bool launch_prefill(const PrefillArgs &a, cudaStream_t s);
 
 }  // namespace kvq

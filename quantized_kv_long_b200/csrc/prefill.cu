@@ -51,7 +51,7 @@
 // Every mbarrier wait is bounded; a wait that runs out records
 // KVQ_ERR_TIMEOUT in the status word and the roles fall through, waiting
 // (bounded) for their own copies and MMAs before the CTA frees TMEM and exits.
-#include <stdlib.h>
+#include <mutex>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -278,7 +278,10 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.n_q_heads / a.n_kv_heads;
     const int rows_total = a.T * G;
-    const int h = blockIdx.y, layer = blockIdx.z;
+    // (layer, KV head) pair of this CTA; `slab` indexes its key tiles in the workspace
+    const int slab = blockIdx.y + blockIdx.z * gridDim.y;
+    const int pair = a.pair0 + slab;
+    const int h = pair % a.n_kv_heads, layer = pair / a.n_kv_heads;
     const int R0 = row0 + blockIdx.x * BM;                 // first row of this tile
     const int r_last = min(R0 + BM, rows_total) - 1;
     const int64_t n_keys = a.n_cached + r_last / G + 1;    // keys any row of the tile sees
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
     const uint8_t *vg = a.layers.v[layer] + (int64_t)h * cap * VROW;
     volatile int *abort = &hd.abort;
     // test hook: the first CTA's producer waits on a barrier that nothing completes
-    const bool hook_wait = a.test_timeout && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+    const bool hook_wait = a.test_timeout && blockIdx.x == 0 && pair == 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NR; ++i) {
@@ -582,7 +585,7 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         if (lane == 0) {
             const int tiles_total = (int)((a.n_cached + a.T + BN - 1) / BN);
             const uint8_t *wsb = static_cast<const uint8_t *>(a.workspace) +
-                                 ((int64_t)layer * a.n_kv_heads + h) * tiles_total * TILE3;
+                                 (int64_t)slab * tiles_total * TILE3;
             int issued = 0;
             for (int j = 0; j < ntiles; ++j) {
                 const int kb = slot(j, NB);
@@ -749,11 +752,14 @@ __global__ void __launch_bounds__(EXP_THREADS) prefill_expand_kernel(const Prefi
     uint8_t *rk = smem + TILE3, *rv = rk + RAW_K;
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + TILE3 + RAW_BYTES);
     __shared__ int ok_s;
-    const int t = blockIdx.x, h = blockIdx.y, layer = blockIdx.z;
+    const int t = blockIdx.x;
+    const int slab = blockIdx.y + blockIdx.z * gridDim.y;  // as in prefill_tc_kernel
+    const int pair = a.pair0 + slab;
+    const int h = pair % a.n_kv_heads, layer = pair / a.n_kv_heads;
     const int64_t n_keys = a.n_cached + a.T;
     const int rows = (int)min((int64_t)BN, n_keys - (int64_t)t * BN);
     const int64_t cap = a.layers.cap[layer];
-    if (threadIdx.x == 0 && a.test_timeout && t == 0 && h == 0 && layer == 0) {
+    if (threadIdx.x == 0 && a.test_timeout && t == 0 && pair == 0) {
         // test hook: a bounded wait on a barrier that nothing completes, before any copy
         ptx::mbar_init(bar, 1);
         ptx::fence_mbar_init();
@@ -762,7 +768,7 @@ __global__ void __launch_bounds__(EXP_THREADS) prefill_expand_kernel(const Prefi
             report_timeout(a.status);
         ok_s = 0;
     }
-    if (a.test_timeout && t == 0 && h == 0 && layer == 0) {
+    if (a.test_timeout && t == 0 && pair == 0) {
         __syncthreads();
         return;
     }
@@ -794,7 +800,7 @@ __global__ void __launch_bounds__(EXP_THREADS) prefill_expand_kernel(const Prefi
     __syncthreads();
     if (threadIdx.x == 0) {
         uint8_t *dst = static_cast<uint8_t *>(a.workspace) +
-                       (((int64_t)layer * a.n_kv_heads + h) * tiles_total + t) * TILE3;
+                       ((int64_t)slab * tiles_total + t) * TILE3;
         ptx::bulk_s2g(dst, smem, TILE3);
         ptx::bulk_commit();
         ptx::bulk_wait_read0();  // the shared memory stays valid until it has been read
@@ -965,14 +971,47 @@ size_t prefill_expand_bytes(int n_layers, int n_kv_heads, int head_dim, int64_t 
     return (size_t)n_layers * n_kv_heads * (size_t)((n_keys + BN - 1) / BN) * TILE3;
 }
 
+size_t prefill_slab_bytes(int head_dim, int64_t n_keys)
+{
+    return prefill_expand_bytes(1, 1, head_dim, n_keys);
+}
+
 bool prefill_supported(int n_q_heads, int n_kv_heads, int head_dim)
 {
     const int G = n_q_heads / n_kv_heads;
     return G >= 1 && G <= 32 && head_dim >= 32 && head_dim <= 512 && head_dim % 32 == 0;
 }
 
-void launch_prefill(const PrefillArgs &a, cudaStream_t s)
+namespace {
+
+// A second stream and two events per device for the double-buffered expansion;
+// the mutex keeps one call's fork and join (which reuse the events) together.
+struct ForkStream {
+    std::mutex mu;
+    cudaStream_t s2 = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+ForkStream g_fork[MAX_DEVICES];
+
+// Expansion and tensor-core attention of the pairs [p0, p0 + np) with their key
+// tiles at `ws` (np slabs).
+void expand_and_attend(PrefillArgs a, int p0, int np, void *ws, int tiles_total, int row0,
+                       int rows, cudaStream_t s)
 {
+    a.pair0 = p0;
+    a.workspace = ws;
+    dim3 egrid((unsigned)tiles_total, (unsigned)np, 1);
+    dim3 grid((unsigned)((rows + BM - 1) / BM), (unsigned)np, 1);
+    prefill_expand_kernel<<<egrid, EXP_THREADS, EXP_SMEM, s>>>(a, tiles_total);
+    prefill_tc_kernel<true><<<grid, pf_threads<true>(), pf_smem<true>(), s>>>(a, row0);
+}
+
+}  // namespace
+
+bool launch_prefill(const PrefillArgs &a_in, cudaStream_t s)
+{
+    PrefillArgs a = a_in;
+    a.pair0 = 0;
     const int G = a.n_q_heads / a.n_kv_heads;
     // tokens whose rows see fewer than PF_MIN_KEYS keys take the exact kernel; so do
     // all rows when per-page partials are asked for (a page is a short context, where
@@ -992,30 +1031,71 @@ void launch_prefill(const PrefillArgs &a, cudaStream_t s)
         dim3 grid((unsigned)((t_split + tb - 1) / tb), a.n_kv_heads, a.n_layers);
         prefill_exact_kernel<<<grid, EX_THREADS, smem, s>>>(a, tb, (int)t_split);
     }
-    if (t_split < a.T) {
-        // with a workspace (the caller checked its size), expand the f16 tiles once
-        const bool pre = a.workspace != nullptr;
-        static std::atomic<int> smem_tc[2][MAX_DEVICES], smem_exp[MAX_DEVICES];
-        if (pre) {
-            ensure_smem(reinterpret_cast<const void *>(prefill_tc_kernel<true>), smem_tc[1],
-                        pf_smem<true>());
-            ensure_smem(reinterpret_cast<const void *>(prefill_expand_kernel), smem_exp, EXP_SMEM);
-        } else {
-            ensure_smem(reinterpret_cast<const void *>(prefill_tc_kernel<false>), smem_tc[0],
-                        pf_smem<false>());
-        }
-        const int row0 = (int)t_split * G;
-        const int rows = a.T * G - row0;
-        dim3 grid((unsigned)((rows + BM - 1) / BM), a.n_kv_heads, a.n_layers);
-        if (pre) {
-            const int tiles_total = (int)((a.n_cached + a.T + BN - 1) / BN);
-            dim3 egrid((unsigned)tiles_total, a.n_kv_heads, a.n_layers);
-            prefill_expand_kernel<<<egrid, EXP_THREADS, EXP_SMEM, s>>>(a, tiles_total);
-            prefill_tc_kernel<true><<<grid, pf_threads<true>(), pf_smem<true>(), s>>>(a, row0);
-        } else {
-            prefill_tc_kernel<false><<<grid, pf_threads<false>(), pf_smem<false>(), s>>>(a, row0);
-        }
+    if (t_split == a.T)
+        return true;
+    const bool pre = a.workspace != nullptr;
+    static std::atomic<int> smem_tc[2][MAX_DEVICES], smem_exp[MAX_DEVICES];
+    if (pre) {
+        ensure_smem(reinterpret_cast<const void *>(prefill_tc_kernel<true>), smem_tc[1],
+                    pf_smem<true>());
+        ensure_smem(reinterpret_cast<const void *>(prefill_expand_kernel), smem_exp, EXP_SMEM);
+    } else {
+        ensure_smem(reinterpret_cast<const void *>(prefill_tc_kernel<false>), smem_tc[0],
+                    pf_smem<false>());
     }
+    const int row0 = (int)t_split * G;
+    const int rows = a.T * G - row0;
+    if (!pre) {
+        dim3 grid((unsigned)((rows + BM - 1) / BM), a.n_kv_heads, a.n_layers);
+        prefill_tc_kernel<false><<<grid, pf_threads<false>(), pf_smem<false>(), s>>>(a, row0);
+        return true;
+    }
+    // With a workspace (the caller checked that it holds at least one slab): every
+    // (layer, KV head) pair's key tiles are expanded once into a slab of it, then read
+    // by all row tiles of the pair.  If every pair has a slab, one expansion and one
+    // attention launch cover the call.  Otherwise the pairs go in chunks through two
+    // halves of the workspace, alternating between the caller's stream and a second
+    // one, so that a chunk's expansion and the start of its attention overlap the end
+    // of the previous chunk's attention.
+    const int tiles_total = (int)((a.n_cached + a.T + BN - 1) / BN);
+    const size_t slab = (size_t)tiles_total * TILE3;
+    const int pairs = a.n_layers * a.n_kv_heads;
+    const int64_t slots = (int64_t)(a.ws_bytes / slab);
+    if (slots >= pairs) {
+        dim3 egrid((unsigned)tiles_total, a.n_kv_heads, a.n_layers);
+        dim3 grid((unsigned)((rows + BM - 1) / BM), a.n_kv_heads, a.n_layers);
+        prefill_expand_kernel<<<egrid, EXP_THREADS, EXP_SMEM, s>>>(a, tiles_total);
+        prefill_tc_kernel<true><<<grid, pf_threads<true>(), pf_smem<true>(), s>>>(a, row0);
+        return true;
+    }
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES)
+        return false;
+    ForkStream &f = g_fork[dev];
+    std::lock_guard<std::mutex> lock(f.mu);
+    if (slots >= 2 && !f.s2) {
+        if (cudaStreamCreateWithFlags(&f.s2, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&f.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&f.join, cudaEventDisableTiming) != cudaSuccess)
+            return false;
+    }
+    if (slots < 2) {  // one slab: the pairs one at a time on the caller's stream
+        for (int p = 0; p < pairs; ++p)
+            expand_and_attend(a, p, 1, ws, tiles_total, row0, rows, s);
+        return true;
+    }
+    const int chunk = (int)(slots / 2);
+    if (cudaEventRecord(f.fork, s) != cudaSuccess ||
+        cudaStreamWaitEvent(f.s2, f.fork, 0) != cudaSuccess)
+        return false;
+    for (int p0 = 0, i = 0; p0 < pairs; p0 += chunk, ++i) {
+        const int np = min(chunk, pairs - p0);
+        expand_and_attend(a, p0, np, ws + (size_t)(i & 1) * chunk * slab, tiles_total, row0,
+                          rows, (i & 1) ? f.s2 : s);
+    }
+    return cudaEventRecord(f.join, f.s2) == cudaSuccess &&
+           cudaStreamWaitEvent(s, f.join, 0) == cudaSuccess;
 }
 
 }  // namespace kvq

@@ -224,13 +224,15 @@ def test_block_format_validation(kvq):
 
 
 def test_prefill_workspace_validation(kvq):
-    """The optional prefill workspace: its size for the expanded f16 key tiles, and a
-    too-small or misaligned one refused before anything is launched."""
+    """The optional prefill workspace: its size for the expanded f16 key tiles (one
+    slab per (layer, KV head) pair), and one smaller than a slab or misaligned
+    refused before anything is launched."""
     nb = kvq.kvq_prefill_workspace_bytes(16, 4, 256, 264192)
     assert nb == 16 * 4 * 8256 * 49152
+    assert kvq.kvq_prefill_workspace_bytes(1, 1, 256, 264192) == 8256 * 49152  # one slab
     assert kvq.kvq_prefill_workspace_bytes(1, 4, 128, 1000) == 0  # no tensor-core path
     L = _layer(kvq, capacity=4096)
-    need = kvq.kvq_prefill_workspace_bytes(1, 4, 256, 1024 + 128)
+    need = kvq.kvq_prefill_workspace_bytes(1, 1, 256, 1024 + 128)
     args = (L, A, 24, 128, 1024, 1024, 1 / 16, A, A)
     _raises(kvq, kvq.KVQ_ERR_WORKSPACE, kvq.kvq_prefill_attn, *args, workspace=A,
             ws_bytes=need - 1)

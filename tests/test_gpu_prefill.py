@@ -93,9 +93,10 @@ def test_prefill262k_full_size_sampled(kvq):
     kvq.kvq_prefill_attn(cache.layers(), qd, Hq, T, nc, w.page, w.scale, out, lse)
     kvq.kvq_check()
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
-    # the launch the benchmark times: with the expanded-tile workspace (26 GB), same bits
-    nb = kvq.kvq_prefill_workspace_bytes(w.n_layers, w.n_kv_heads, 256, nc + T)
-    ws = torch.empty((nb,), dtype=torch.uint8, device=device)
+    # the launch the benchmark times: a 2 GiB workspace (four of the 64 slabs, two
+    # pairs per chunk), same bits
+    slab = kvq.kvq_prefill_workspace_bytes(1, 1, 256, nc + T)
+    ws = torch.empty(((2 << 30) // slab * slab,), dtype=torch.uint8, device=device)
     out2 = torch.full_like(out, float("nan"))
     lse2 = torch.full_like(lse, float("nan"))
     kvq.kvq_prefill_attn(cache.layers(), qd, Hq, T, nc, w.page, w.scale, out2, lse2, workspace=ws)
@@ -112,6 +113,36 @@ def test_prefill262k_full_size_sampled(kvq):
                                   w.scale)
         assert_attn_close(out[l, ts, hs].cpu().numpy(), lse[l, ts, hs].cpu().numpy(), ro, rl,
                           f"prefill262k layer {l}")
+
+
+@pytest.mark.parametrize("slabs", [1, 2, 3, 5, 7])
+def test_bounded_workspace_chunks_bit_identical(kvq, slabs):
+    """A workspace of fewer slabs than (layer, KV head) pairs (2 layers x 4 heads = 8):
+    one slab runs the pairs one at a time; more alternate chunks of slabs // 2 pairs
+    between two streams.  Every size gives the bits of the full workspace."""
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=16448, T=64)
+    T, nc, L = 64, 16448, 2
+    n = nc + T
+    cache, _ = fill_both(w, list(range(L)), n, -(-n // 8) * 8)
+    q = torch.from_numpy(np.stack([wl.q_rows(w, l, T) for l in range(L)])).cuda()
+    Hq, D = w.n_q_heads, w.head_dim
+    slab = kvq.kvq_prefill_workspace_bytes(1, 1, D, n)
+    assert kvq.kvq_prefill_workspace_bytes(L, w.n_kv_heads, D, n) == 8 * slab
+
+    def run(nbytes):
+        out = torch.full((L, T, Hq, D), float("nan"), device="cuda")
+        lse = torch.full((L, T, Hq), float("nan"), device="cuda")
+        ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device="cuda")
+        kvq.kvq_prefill_attn(cache.layers(), q, Hq, T, nc, 1024, w.scale, out, lse, workspace=ws)
+        kvq.kvq_check()
+        return out, lse
+
+    ref_out, ref_lse = run(8 * slab)
+    out, lse = run(slabs * slab + 256)
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+    with pytest.raises(kvq.KvqError) as e:
+        run(slab - 256)
+    assert e.value.status == kvq.KVQ_ERR_WORKSPACE
 
 
 @pytest.mark.parametrize("Hq,H,n_cached,T,page", [
