@@ -48,6 +48,9 @@ from quantized_kv_long_b200 import workload as wl  # noqa: E402
 METRIC = "q8_0/q4_0 decode attn: KV GB/s (% of HBM peak), query-tok/s at 262k ctx"
 FALLBACK_HBM_GBS = 6650.0
 KV_BYTES_PER_TOKEN_LAYER = lambda w: w.n_kv_heads * (w.head_dim // 32) * (34 + 18)  # noqa: E731
+# --kv-formats: (K block type, V block type) of the C ABI and the bytes of one block of each
+KV_FORMATS = {"q8_0/q4_0": (1, 2, 34, 18), "q8_0/q8_0": (1, 1, 34, 34),
+              "q4_0/q4_0": (2, 2, 18, 18), "q4_0/q8_0": (2, 1, 18, 34)}
 
 
 # --------------------------------------------------------------------------- helpers
@@ -175,10 +178,11 @@ def traffic_record(kernel_files: tuple[str, ...], record: str = "decode_traffic.
 
 # --------------------------------------------------------------------------- our arm
 
-def fill_cache(kvq, torch, w: wl.Workload, device):
+def fill_cache(kvq, torch, w: wl.Workload, device, k_type: int = 0, v_type: int = 0):
     """Quantize the whole context of every layer into a device cache (setup,
     untimed): rows [0, n_kv) drawn per layer by the seeded generator."""
-    cache = kvq.QuantizedKVCache(w.n_layers, w.n_kv_heads, w.head_dim, w.capacity, device=device)
+    cache = kvq.QuantizedKVCache(w.n_layers, w.n_kv_heads, w.head_dim, w.capacity, device=device,
+                                 k_type=k_type, v_type=v_type)
     for l in range(w.n_layers):
         for start in range(0, w.n_kv, 131072):
             stop = min(w.n_kv, start + 131072)
@@ -204,7 +208,8 @@ def run_ours(args, w: wl.Workload) -> dict | None:
     L, T, Hq, D, n_kv, chunk = w.n_layers, w.T, w.n_q_heads, w.head_dim, w.n_kv, w.chunk
     C = w.n_chunks
     rows = L * T * Hq
-    cache = fill_cache(kvq, torch, w, device)
+    k_type, v_type, k_blk, v_blk = KV_FORMATS[args.kv_formats]
+    cache = fill_cache(kvq, torch, w, device, k_type, v_type)
     layers = cache.layers()
     # the step's inputs: q and the T new rows of every layer (rows n_kv-T .. n_kv-1)
     q_h = np.stack([wl.q_rows(w, l) for l in range(L)])
@@ -286,22 +291,24 @@ def run_ours(args, w: wl.Workload) -> dict | None:
     # sanity: outputs are finite (the parity tests check them against the oracle)
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
 
-    kv_bytes = L * n_kv * KV_BYTES_PER_TOKEN_LAYER(w)
+    kv_bytes = L * n_kv * w.n_kv_heads * (D // 32) * (k_blk + v_blk)
     peak, peak_kind = peaks()
     cl = clocks.summary()
     res = None
     if rank == 0:
         gbs = weak_gbs(world, kv_bytes, ms)
         achieved = kv_bytes / (dec_ms_max * 1e-3) / 1e9
-        tr = traffic_record(DECODE_SOURCES)
+        tr = traffic_record(DECODE_SOURCES) if args.kv_formats == "q8_0/q4_0" else None
+        kf, vf = args.kv_formats.split("/")
         res = {
             "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "q8_0 K / q4_0 V x f16 q, f32 accumulate", "data": "synthetic",
+            "dtype": f"{kf} K / {vf} V x f16 q, f32 accumulate", "data": "synthetic",
             "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": w.n_kv_heads,
                        "head_dim": D, "context": n_kv, "query_tokens": T, "chunk": chunk,
                        "seed": w.seed, "kv_bytes_per_step": kv_bytes,
+                       "kv_formats": args.kv_formats,
                        "l2": "inputs larger than L2 (7 GB cache vs 126 MB)",
                        "step": "append, decode, merge: 3 launches",
                        "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
@@ -661,6 +668,9 @@ def main(argv=None) -> int:
     ap.add_argument("--config", default="verify262k",
                     choices=["verify262k", "decode65k", "tiny", "prefill262k", "stream262k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-formats", choices=sorted(KV_FORMATS), default="q8_0/q4_0",
+                    help="decode configs: block formats of K and V (the other pairs run the "
+                         "general decode kernel)")
     ap.add_argument("--ws-mib", type=int, default=2048,
                     help="prefill262k: workspace for the expanded key tiles, MiB (whole slabs "
                          "of one (layer, KV head) each; 0 = one slab per pair, 26 GB)")

@@ -284,9 +284,8 @@ kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k
  *            the same results bit for bit.  Ignored when the tensor-core path
  *            does not run.  Owned by the caller; not used after the call's
  *            work completes.
- * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (group size > 32, block formats
- *         other than Q8_0 K / Q4_0 V), WORKSPACE (a workspace smaller than one
- *         slab), CUDA. */
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (group size > 32),
+ *         WORKSPACE (a workspace smaller than one slab), CUDA. */
 kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
                             int n_q_heads, int T, int64_t n_cached, int page, float scale,
                             float *out, float *lse, float *page_out, float *page_lse,

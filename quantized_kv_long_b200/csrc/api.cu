@@ -372,8 +372,6 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
     if (!prefill_supported(n_q_heads, H, D))
         return set_error(KVQ_ERR_UNSUPPORTED, "%s: head_dim=%d, group=%d not supported", fn, D,
                          n_q_heads / H);
-    if (k_type_of(layers[0]) != KVQ_TYPE_Q8_0 || v_type_of(layers[0]) != KVQ_TYPE_Q4_0)
-        return set_error(KVQ_ERR_UNSUPPORTED, "%s: only Q8_0 K with Q4_0 V is implemented", fn);
     const size_t ws = prefill_workspace_bytes(n_layers, n_q_heads, H, T, D);
     if (ws > 0 && (workspace == nullptr || ws_bytes < ws))
         return set_error(KVQ_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn,
@@ -395,6 +393,8 @@ kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_
     a.lse = lse;
     a.page_out = page_out;
     a.page_lse = page_lse;
+    a.k_type = k_type_of(layers[0]);
+    a.v_type = v_type_of(layers[0]);
     // optional workspace: the f16 key tiles of the tensor-core path, expanded once
     a.workspace = nullptr;
     a.ws_bytes = 0;

@@ -21,6 +21,23 @@ __host__ __device__ inline int64_t v_row_bytes(int head_dim) { return (int64_t)(
 // Block formats (kvq_type resolved: KVQ_TYPE_DEFAULT becomes Q8_0 for K, Q4_0 for V).
 __host__ __device__ inline int block_bytes(int type) { return type == KVQ_TYPE_Q8_0 ? Q8_0_BYTES : Q4_0_BYTES; }
 __host__ __device__ inline int64_t row_bytes(int type, int head_dim) { return (int64_t)(head_dim / QK) * block_bytes(type); }
+
+// Integer value of element i (0..31) of a block: int8 q (Q8_0) or nibble - 8
+// (Q4_0: byte i holds element i in the low nibble and element i + 16 in the high).
+template <int TYPE>
+__device__ __forceinline__ int block_int(const uint8_t *blk, int i)
+{
+    if (TYPE == KVQ_TYPE_Q8_0)
+        return (int)(int8_t)blk[2 + i];
+    const uint8_t byte = blk[2 + (i & 15)];
+    return (i < 16 ? (byte & 15) : (byte >> 4)) - 8;
+}
+
+// The block's fp16 scale d (first two bytes, little-endian) as fp32.
+__device__ __forceinline__ float block_d(const uint8_t *blk)
+{
+    return __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
+}
 inline int k_type_of(const kvq_layer &l) { return l.k_type ? l.k_type : KVQ_TYPE_Q8_0; }
 inline int v_type_of(const kvq_layer &l) { return l.v_type ? l.v_type : KVQ_TYPE_Q4_0; }
 
@@ -127,6 +144,7 @@ struct PrefillArgs {
     unsigned int *status;
     int test_timeout;  // test hook: one bounded wait of each tensor-core launch runs out
     int pair0;         // first (layer, KV head) pair, layer * n_kv_heads + head, of a launch
+    int k_type, v_type;  // block formats (KVQ_TYPE_Q8_0 / KVQ_TYPE_Q4_0)
 };
 size_t prefill_workspace_bytes(int n_layers, int n_q_heads, int n_kv_heads, int T, int head_dim);
 // Optional workspace of the tensor-core path: the f16 key tiles expanded once per

@@ -23,22 +23,6 @@ namespace kvq {
 constexpr int SIMPLE_THREADS = 256;
 constexpr int SIMPLE_TILE = 64;
 
-// Integer value of element i (0..31) of a block: int8 q (Q8_0) or nibble - 8
-// (Q4_0: byte i holds element i in the low nibble and element i + 16 in the high).
-template <int TYPE>
-__device__ __forceinline__ int block_int(const uint8_t *blk, int i)
-{
-    if (TYPE == KVQ_TYPE_Q8_0)
-        return (int)(int8_t)blk[2 + i];
-    const uint8_t byte = blk[2 + (i & 15)];
-    return (i < 16 ? (byte & 15) : (byte >> 4)) - 8;
-}
-
-__device__ __forceinline__ float block_d(const uint8_t *blk)
-{
-    return __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
-}
-
 template <int KT, int VT>
 __global__ void __launch_bounds__(SIMPLE_THREADS)
 decode_simple_kernel(DecodeArgs a)

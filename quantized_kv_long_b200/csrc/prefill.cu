@@ -813,6 +813,7 @@ __global__ void __launch_bounds__(EXP_THREADS) prefill_expand_kernel(const Prefi
 // softmax in fp32; per-block K scale applied to each block's fp32 dot product.
 constexpr int EX_THREADS = 256, EX_TILE = 64;
 
+template <int KT, int VT>
 __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const PrefillArgs a, int tb_tok,
                                                                    int t_end)
 {
@@ -829,8 +830,9 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
     float *m_s = p_s + R * EX_TILE;
     float *l_s = m_s + R;
     float *al_s = l_s + R;
-    const uint8_t *kb = a.layers.k[layer] + (int64_t)h * a.layers.cap[layer] * k_row_bytes(D);
-    const uint8_t *vb = a.layers.v[layer] + (int64_t)h * a.layers.cap[layer] * v_row_bytes(D);
+    const int64_t krow = row_bytes(KT, D), vrow = row_bytes(VT, D);
+    const uint8_t *kb = a.layers.k[layer] + (int64_t)h * a.layers.cap[layer] * krow;
+    const uint8_t *vb = a.layers.v[layer] + (int64_t)h * a.layers.cap[layer] * vrow;
     for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
         const int r = p / D, i = p % D;
         const int t = t0 + r / G, g = r % G;
@@ -877,16 +879,15 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
             const int t = t0 + r / G;
             float s = -INFINITY;
             if (j <= a.n_cached + t) {
-                const uint8_t *kr = kb + j * k_row_bytes(D);
+                const uint8_t *kr = kb + j * krow;
                 const float *qr = q_s + r * D;
                 float tot = 0.0f;
                 for (int bq = 0; bq < nb; ++bq) {
-                    const uint8_t *blk = kr + bq * Q8_0_BYTES;
-                    const float d = __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
+                    const uint8_t *blk = kr + bq * block_bytes(KT);
                     float part = 0.0f;
                     for (int i = 0; i < QK; ++i)
-                        part += qr[bq * QK + i] * (float)(int8_t)blk[2 + i];
-                    tot += d * part;
+                        part += qr[bq * QK + i] * (float)block_int<KT>(blk, i);
+                    tot += block_d(blk) * part;
                 }
                 s = a.scale * tot;
             }
@@ -924,11 +925,8 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
                 const float pw = p_s[r * EX_TILE + jj];
                 if (pw == 0.0f)
                     continue;
-                const uint8_t *blk = vb + (j0 + jj) * v_row_bytes(D) + bq * Q4_0_BYTES;
-                const float d = __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
-                const uint8_t byte = blk[2 + (ii & 15)];
-                const int u = ii < 16 ? (byte & 15) : (byte >> 4);
-                o += pw * (d * (float)(u - 8));
+                const uint8_t *blk = vb + (j0 + jj) * vrow + bq * block_bytes(VT);
+                o += pw * (block_d(blk) * (float)block_int<VT>(blk, ii));
             }
             acc[p] = o;
         }
@@ -993,6 +991,14 @@ struct ForkStream {
 };
 ForkStream g_fork[MAX_DEVICES];
 
+template <int KT, int VT>
+void launch_exact(const PrefillArgs &a, dim3 grid, size_t smem, int tb, int t_end, cudaStream_t s)
+{
+    static std::atomic<int> smem_ex[MAX_DEVICES];
+    ensure_smem(reinterpret_cast<const void *>(prefill_exact_kernel<KT, VT>), smem_ex, (int)smem);
+    prefill_exact_kernel<KT, VT><<<grid, EX_THREADS, smem, s>>>(a, tb, t_end);
+}
+
 // Expansion and tensor-core attention of the pairs [p0, p0 + np) with their key
 // tiles at `ws` (np slabs).
 void expand_and_attend(PrefillArgs a, int p0, int np, void *ws, int tiles_total, int row0,
@@ -1020,16 +1026,23 @@ bool launch_prefill(const PrefillArgs &a_in, cudaStream_t s)
     t_split = t_split < 0 ? 0 : (t_split > a.T ? a.T : t_split);
     if (a.page_out)
         t_split = a.T;
-    if (a.head_dim != HD)
-        t_split = a.T;  // the tensor-core path is built for head_dim 256
+    // the tensor-core path is built for head_dim 256 and Q8_0 K / Q4_0 V
+    if (a.head_dim != HD || a.k_type != KVQ_TYPE_Q8_0 || a.v_type != KVQ_TYPE_Q4_0)
+        t_split = a.T;
     if (t_split > 0) {
         const int tb = max(1, 32 / G);
         const size_t smem = sizeof(float) * ((size_t)2 * tb * G * a.head_dim +
                                              (size_t)tb * G * EX_TILE + 3 * (size_t)tb * G);
-        static std::atomic<int> smem_ex[MAX_DEVICES];
-        ensure_smem(reinterpret_cast<const void *>(prefill_exact_kernel), smem_ex, (int)smem);
         dim3 grid((unsigned)((t_split + tb - 1) / tb), a.n_kv_heads, a.n_layers);
-        prefill_exact_kernel<<<grid, EX_THREADS, smem, s>>>(a, tb, (int)t_split);
+        constexpr int Q8 = KVQ_TYPE_Q8_0, Q4 = KVQ_TYPE_Q4_0;
+        if (a.k_type == Q8 && a.v_type == Q4)
+            launch_exact<Q8, Q4>(a, grid, smem, tb, (int)t_split, s);
+        else if (a.k_type == Q8 && a.v_type == Q8)
+            launch_exact<Q8, Q8>(a, grid, smem, tb, (int)t_split, s);
+        else if (a.k_type == Q4 && a.v_type == Q4)
+            launch_exact<Q4, Q4>(a, grid, smem, tb, (int)t_split, s);
+        else
+            launch_exact<Q4, Q8>(a, grid, smem, tb, (int)t_split, s);
     }
     if (t_split == a.T)
         return true;

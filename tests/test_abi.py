@@ -205,8 +205,8 @@ def test_resident_layers_plan(kvq):
 
 
 def test_block_format_validation(kvq):
-    """Block formats: unknown types and layers that differ are refused; prefill
-    implements the default pair only; the residency plan sizes layers by format."""
+    """Block formats: unknown types and layers that differ are refused (prefill
+    included); the residency plan sizes layers by format."""
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, _layer(kvq, k_type=3), A, A, 0, 1, 0)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, _layer(kvq, v_type=-1), A, A, 0, 1, 0)
     # explicit Q8_0 K / Q4_0 V equals the default pair, so these two layers agree
@@ -215,7 +215,8 @@ def test_block_format_validation(kvq):
             A, A, 0, 1, 0)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_decode_attn,
             [_layer(kvq, k_type=2), _layer(kvq)], A, 24, 1, 1024, 256, 1 / 16, A, A, 0)
-    _raises(kvq, kvq.KVQ_ERR_UNSUPPORTED, kvq.kvq_prefill_attn, _layer(kvq, v_type=1, capacity=4096),
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_prefill_attn,
+            [_layer(kvq, v_type=1, capacity=4096), _layer(kvq, capacity=4096)],
             A, 24, 128, 1024, 1024, 1 / 16, A, A)
     q8 = 4 * 262144 * (272 + 272)
     assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 1, 1) == 3

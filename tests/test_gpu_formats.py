@@ -4,8 +4,8 @@ choices of the KV-cache guide's levers section) on the GPU, against the oracle.
 The default pair (Q8_0 K / Q4_0 V) is covered by the other GPU tests; here
 the three other pairs go through append (bit-exact cache bytes), the general
 decode kernel and the merge (tolerances of helpers.py), the decode step
-(three launches for these formats, bit-identical to the separate calls) and
-the streamed decode (bit-identical to the resident one).
+(bit-identical to the separate calls), the streamed decode (bit-identical to
+the resident one) and prefill (the exact kernel, which serves every pair).
 """
 import numpy as np
 import pytest
@@ -119,3 +119,23 @@ def test_streamed_q8_0_values(kvq):
         kvq.kvq_merge_lse(op2, lp2, T * Hq, C, D, o2, l2)
         kvq.kvq_check()
         assert torch.equal(out[l], o2) and torch.equal(lse[l], l2)
+
+
+@pytest.mark.parametrize("k_type,v_type", PAIRS)
+def test_prefill_formats(kvq, k_type, v_type):
+    """Prefill on these formats: every row on the exact kernel (the tensor-core path
+    is built for Q8_0 K / Q4_0 V), 2 layers, rows seeing 16,100 to 16,139 keys."""
+    n_cached, T, L = 16100, 40, 2
+    n = n_cached + T
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=n_cached, T=T)
+    cache, orc = fill_both(w, list(range(L)), n, -(-n // 8) * 8, k_type=k_type, v_type=v_type)
+    q = q_all(w, list(range(L)), T)
+    Hq, D = w.n_q_heads, w.head_dim
+    out = torch.full((L, T, Hq, D), float("nan"), device="cuda")
+    lse = torch.full((L, T, Hq), float("nan"), device="cuda")
+    kvq.kvq_prefill_attn(cache.layers(), torch.from_numpy(q).cuda(), Hq, T, n_cached, 4096,
+                         w.scale, out, lse)
+    kvq.kvq_check()
+    for l in range(L):
+        ro, rl = oracle.prefill_attn(orc[l][0], orc[l][1], q[l], n_cached, 4096, w.scale)
+        assert_attn_close(out[l].cpu().numpy(), lse[l].cpu().numpy(), ro, rl, f"layer {l}")

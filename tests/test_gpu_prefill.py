@@ -194,3 +194,18 @@ def test_prefill_bounded_wait_times_out_and_context_survives(kvq, expand):
     out, lse = run_prefill(kvq, cache, q, w.n_q_heads, T, n_cached, w.scale, expand=expand)
     ro, rl = oracle.prefill_attn(orc[0][0], orc[0][1], q[0], n_cached, 1024, w.scale)
     assert_attn_close(out[0], lse[0], ro, rl, "after timeout")
+
+
+@pytest.mark.parametrize("Hq,H,D,n_cached,T", [
+    (8, 2, 512, 3000, 24),       # head_dim 512: the exact kernel (tensor cores need 256)
+    (4, 4, 256, 16400, 160),     # G = 1: 160 rows per head, tensor cores, ragged tile
+    (16, 2, 256, 16350, 48),     # G = 8: exact rows (t < 34) then tensor-core rows
+    (32, 1, 256, 16448, 8),      # G = 32: one 256-row head, two row tiles
+    (32, 1, 128, 500, 6),        # G = 32 at head_dim 128 on the exact kernel
+])
+def test_head_dims_and_group_sizes(kvq, Hq, H, D, n_cached, T):
+    """Other head_dims and GQA ratios against the oracle, with the workspace path
+    bit-identical to the in-CTA dequantization where the tensor cores run."""
+    w = wl.small(wl.WORKLOADS["prefill262k"], n_cached=n_cached, T=T, n_q_heads=Hq,
+                 n_kv_heads=H, head_dim=D)
+    check(kvq, w, 1, T, n_cached)
