@@ -43,6 +43,7 @@ if ROOT not in sys.path:
 
 import numpy as np  # noqa: E402
 
+from quantized_kv_long_b200 import context_parallel as cp  # noqa: E402
 from quantized_kv_long_b200 import workload as wl  # noqa: E402
 
 METRIC = "q8_0/q4_0 decode attn: KV GB/s (% of HBM peak), query-tok/s at 262k ctx"
@@ -178,17 +179,21 @@ def traffic_record(kernel_files: tuple[str, ...], record: str = "decode_traffic.
 
 # --------------------------------------------------------------------------- our arm
 
-def fill_cache(kvq, torch, w: wl.Workload, device, k_type: int = 0, v_type: int = 0):
-    """Quantize the whole context of every layer into a device cache (setup,
-    untimed): rows [0, n_kv) drawn per layer by the seeded generator."""
-    cache = kvq.QuantizedKVCache(w.n_layers, w.n_kv_heads, w.head_dim, w.capacity, device=device,
+def fill_cache(kvq, torch, w: wl.Workload, device, k_type: int = 0, v_type: int = 0,
+               key0: int = 0, n_keys: int | None = None):
+    """Quantize the context of every layer into a device cache (setup, untimed):
+    keys [key0, key0 + n_keys) (default: all n_kv) drawn per layer by the seeded
+    generator, at cache rows [0, n_keys)."""
+    n_keys = w.n_kv if n_keys is None else n_keys
+    cap = w.capacity if (key0, n_keys) == (0, w.n_kv) else -(-n_keys // 8) * 8
+    cache = kvq.QuantizedKVCache(w.n_layers, w.n_kv_heads, w.head_dim, cap, device=device,
                                  k_type=k_type, v_type=v_type)
     for l in range(w.n_layers):
-        for start in range(0, w.n_kv, 131072):
-            stop = min(w.n_kv, start + 131072)
+        for start in range(key0, key0 + n_keys, 131072):
+            stop = min(key0 + n_keys, start + 131072)
             k = torch.from_numpy(wl.kv_rows(w, l, 0, start, stop)).to(device)
             v = torch.from_numpy(wl.kv_rows(w, l, 1, start, stop)).to(device)
-            kvq.kvq_append(cache.layer(l), k, v, start, stop - start)
+            kvq.kvq_append(cache.layer(l), k, v, start - key0, stop - start)
     torch.cuda.synchronize(device)
     return cache
 
@@ -206,11 +211,17 @@ def run_ours(args, w: wl.Workload) -> dict | None:
     stream = torch.cuda.current_stream(device)
 
     L, T, Hq, D, n_kv, chunk = w.n_layers, w.T, w.n_q_heads, w.head_dim, w.n_kv, w.chunk
-    C = w.n_chunks
     rows = L * T * Hq
     k_type, v_type, k_blk, v_blk = KV_FORMATS[args.kv_formats]
-    cache = fill_cache(kvq, torch, w, device, k_type, v_type)
+    # --split context: this rank holds keys [key0, key0 + n_keys) of every layer and the
+    # ranks exchange their merged rows; replicas: every rank holds the whole context
+    split = args.split == "context"
+    key0, n_keys = cp.shard_range(n_kv, world, rank, chunk) if split else (0, n_kv)
+    C = -(-n_keys // chunk)
+    cache = fill_cache(kvq, torch, w, device, k_type, v_type, key0, n_keys)
     layers = cache.layers()
+    # the new rows [n_kv - T, n_kv) that fall in this rank's keys
+    a0, a1 = max(n_kv - T, key0), min(n_kv, key0 + n_keys)
     # the step's inputs: q and the T new rows of every layer (rows n_kv-T .. n_kv-1)
     q_h = np.stack([wl.q_rows(w, l) for l in range(L)])
     k_h = np.stack([wl.kv_rows(w, l, 0, n_kv - T, n_kv) for l in range(L)])
@@ -222,20 +233,40 @@ def run_ours(args, w: wl.Workload) -> dict | None:
     lp = torch.empty((L, T, Hq, C), device=device)
     out = torch.empty((L, T, Hq, D), device=device)
     lse = torch.empty((L, T, Hq), device=device)
+    exchange = split and world > 1
+    if exchange:
+        out_r = torch.empty((rows, D), device=device)
+        lse_r = torch.empty((rows,), device=device)
 
+        def merge_parts(po, pl, o, l):
+            kvq.kvq_merge_lse_parts(po, pl, world, rows, D, o, l, stream)
+
+    # this rank's part of the new rows (a view when it is all of them; the e2e copies
+    # below refresh k_new / v_new, so a partial part is a view too: rows a0.. of dim 1)
+    k_app = k_new[:, a0 - (n_kv - T):a1 - (n_kv - T)]
+    v_app = v_new[:, a0 - (n_kv - T):a1 - (n_kv - T)]
+    if a1 > a0 and (a0, a1) != (n_kv - T, n_kv):
+        k_app, v_app = k_app.contiguous(), v_app.contiguous()  # [L][a1 - a0][H][D]
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
 
     def step(i=None):
         # append, decode, merge: the three launches of kvq_decode_step, issued one by one
-        # so that the decode launch can be timed on its own
-        kvq.kvq_append(layers, k_new, v_new, n_kv - T, T, stream)
+        # so that the decode launch can be timed on its own (a context split decodes this
+        # rank's shard, merges it, all-gathers the merged rows and merges the ranks')
+        if a1 > a0:
+            kvq.kvq_append(layers, k_app, v_app, a0 - key0, a1 - a0, stream)
         if i is not None:
             ev_dec[i][0].record(stream)
-        kvq.kvq_decode_attn(layers, q, Hq, T, n_kv, chunk, w.scale, op, lp, stream)
+        kvq.kvq_decode_attn_shard(layers, q, Hq, T, n_keys, key0, n_kv, chunk, w.scale, op, lp,
+                                  stream)
         if i is not None:
             ev_dec[i][1].record(stream)
-        kvq.kvq_merge_lse(op, lp, rows, C, D, out, lse, stream)
+        if not exchange:
+            kvq.kvq_merge_lse(op, lp, rows, C, D, out, lse, stream)
+            return
+        kvq.kvq_merge_lse(op, lp, rows, C, D, out_r, lse_r, stream)
+        cp.gather_merge(out_r, lse_r, out.view(rows, D), lse.view(rows), merge_parts)
 
     for _ in range(args.warmup):
         step()
@@ -291,41 +322,53 @@ def run_ours(args, w: wl.Workload) -> dict | None:
     # sanity: outputs are finite (the parity tests check them against the oracle)
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
 
-    kv_bytes = L * n_kv * w.n_kv_heads * (D // 32) * (k_blk + v_blk)
+    tok_bytes = L * w.n_kv_heads * (D // 32) * (k_blk + v_blk)  # one key of every layer
+    kv_bytes = n_kv * tok_bytes    # the context of one replica, or of all ranks when split
+    # a replica reads its whole context; a context split divides one context over the ranks
+    per_rank = weak_gbs(world, kv_bytes, ms) if not split else kv_bytes / (ms * 1e-3) / 1e9
+    e2e_gbs = weak_gbs(world, kv_bytes, e2e_ms) if not split else kv_bytes / (e2e_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
     cl = clocks.summary()
     res = None
     if rank == 0:
-        gbs = weak_gbs(world, kv_bytes, ms)
-        achieved = kv_bytes / (dec_ms_max * 1e-3) / 1e9
-        tr = traffic_record(DECODE_SOURCES) if args.kv_formats == "q8_0/q4_0" else None
+        gbs = per_rank
+        # the decode launch of rank 0 against its own keys (the slowest rank's time)
+        achieved = n_keys * tok_bytes / (dec_ms_max * 1e-3) / 1e9
+        tr = (traffic_record(DECODE_SOURCES)
+              if args.kv_formats == "q8_0/q4_0" and (key0, n_keys) == (0, n_kv) else None)
         kf, vf = args.kv_formats.split("/")
         res = {
             "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if split else "weak",
+            "vs_baseline": None,
             "dtype": f"{kf} K / {vf} V x f16 q, f32 accumulate", "data": "synthetic",
             "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": w.n_kv_heads,
                        "head_dim": D, "context": n_kv, "query_tokens": T, "chunk": chunk,
                        "seed": w.seed, "kv_bytes_per_step": kv_bytes,
                        "kv_formats": args.kv_formats,
                        "l2": "inputs larger than L2 (7 GB cache vs 126 MB)",
-                       "step": "append, decode, merge: 3 launches",
-                       "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
+                       "step": ("append, decode, merge: 3 launches" if not exchange else
+                                "append, decode of the shard, merge, all-gather (NCCL), merge "
+                                "of the ranks' rows"),
+                       "parallelism": (f"context{world}" if split and world > 1 else
+                                       f"replicas{world}" if world > 1 else "single-gpu")},
             # query tokens per step (each attends all L layers) / step time
-            "query_tok_per_s": round(world * T / (ms * 1e-3), 1),
-            "layer_query_tok_per_s": round(world * L * T / (ms * 1e-3), 1),
+            "query_tok_per_s": round((1 if split else world) * T / (ms * 1e-3), 1),
+            "layer_query_tok_per_s": round((1 if split else world) * L * T / (ms * 1e-3), 1),
             "pct_hbm_peak": round(100 * gbs / world / peak, 2),
-            "e2e": {"value": round(weak_gbs(world, kv_bytes, e2e_ms), 1), "unit": "GB/s",
+            "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 4)},
             "roofline": {"bound": "hbm",
-                         "kernel": f"kvq_decode_attn ({L} layers, 1 launch)",
+                         "kernel": (f"kvq_decode_attn ({L} layers, 1 launch)" if not split else
+                                    f"kvq_decode_attn_shard ({L} layers x {n_keys} keys, "
+                                    f"1 launch)"),
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": tr["dram_bytes_per_launch"] if tr else None,
                          "launch_ms": round(dec_ms_max, 4)},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": ((a1 > a0) + 2 + exchange) * args.steps,
             "clocks": {"sm_mhz": cl["sm_mhz"], "sm_max_mhz": cl["sm_max_mhz"],
                        "reasons": cl["reasons"], "samples": cl["samples"]},
         }
@@ -668,6 +711,10 @@ def main(argv=None) -> int:
     ap.add_argument("--config", default="verify262k",
                     choices=["verify262k", "decode65k", "tiny", "prefill262k", "stream262k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", choices=["replicas", "context"], default="replicas",
+                    help="decode configs with N > 1: one replica per GPU (default), or one "
+                         "context split over the GPUs (each decodes its shard of the keys; the "
+                         "merged rows are all-gathered over NCCL and merged)")
     ap.add_argument("--kv-formats", choices=sorted(KV_FORMATS), default="q8_0/q4_0",
                     help="decode configs: block formats of K and V (the other pairs run the "
                          "general decode kernel)")

@@ -188,6 +188,28 @@ kvq_status kvq_decode_attn(const kvq_layer *layers, int n_layers, const uint16_t
                            int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
                            float *out_part, float *lse_part, kvq_stream stream);
 
+/* kvq_decode_attn over one contiguous shard of a context, for a
+ * context-parallel split (each GPU holds keys [key0, key0 + n_keys) of an
+ * n_kv-key context and decodes only those; the shards' results are then
+ * combined by the LSE merge, e.g. kvq_merge_lse followed by an all-gather and
+ * kvq_merge_lse_parts).  The layers hold the shard's keys at their rows
+ * [0, n_keys); query token t sees the global keys j <= n_kv - T + t, i.e. the
+ * shard rows j' <= n_kv - T + t - key0 (a row that sees none of the shard gets
+ * out = 0, lse = -inf).  Chunks split the shard: n_chunks = ceil(n_keys /
+ * chunk).  With key0 = 0 and n_keys = n_kv this is kvq_decode_attn.
+ * Source: as kvq_decode_attn; the split is this library's extension (the
+ * merge that combines the shards is the one the pages use across pages).
+ *  n_keys    keys in the shard, 1 <= n_keys <= capacity
+ *  key0      global index of the shard's first key, 0 <= key0 <= n_kv - n_keys
+ *  n_kv      keys in the whole context (including the T new rows), >= T
+ *  other arguments as kvq_decode_attn, with n_chunks from n_keys
+ * Errors: those of kvq_decode_attn; INVALID_ARG for a shard outside the
+ *         context. */
+kvq_status kvq_decode_attn_shard(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                                 int n_q_heads, int T, int64_t n_keys, int64_t key0,
+                                 int64_t n_kv, int chunk, float scale, float *out_part,
+                                 float *lse_part, kvq_stream stream);
+
 /* ---------------------------------------------------------------------- */
 /* LSE merge                                                               */
 /* ---------------------------------------------------------------------- */
@@ -205,6 +227,19 @@ kvq_status kvq_decode_attn(const kvq_layer *layers, int n_layers, const uint16_t
 kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t rows,
                          int n_chunks, int head_dim, float *out, float *lse,
                          kvq_stream stream);
+
+/* The same merge over partials stored part-major, as an all-gather of
+ * per-rank merged rows lays them out: part p of row r at
+ * out_parts[(p * rows + r) * head_dim ...] and lse_parts[p * rows + r].  The
+ * order of operations is that of kvq_merge_lse (parts in increasing p).
+ *  out_parts device fp32 [n_parts][rows][head_dim], 16-B aligned
+ *  lse_parts device fp32 [n_parts][rows]
+ *  out       device fp32 [rows][head_dim]; lse device fp32 [rows]
+ * Errors: INVALID_ARG (nulls, rows < 0, n_parts < 1, head_dim % 4),
+ *         ALIGNMENT, CUDA. */
+kvq_status kvq_merge_lse_parts(const float *out_parts, const float *lse_parts, int n_parts,
+                               int64_t rows, int head_dim, float *out, float *lse,
+                               kvq_stream stream);
 
 /* ---------------------------------------------------------------------- */
 /* Fused decode step                                                       */

@@ -132,7 +132,8 @@ static void fill_table(const kvq_layer *layers, int n, LayerTable &t)
 // Shared by kvq_decode_attn and kvq_stream_decode.
 kvq_status validate_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
                            int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
-                           const float *out_part, const float *lse_part, const char *fn)
+                           const float *out_part, const float *lse_part, const char *fn,
+                           int64_t min_keys)
 {
     KVQ_TRY(check_layers(layers, n_layers, fn));
     KVQ_TRY(need(q, 16, "q", fn));
@@ -152,8 +153,11 @@ kvq_status validate_decode(const kvq_layer *layers, int n_layers, const uint16_t
     if (chunk < 64 || chunk % 64 != 0)
         return set_error(KVQ_ERR_INVALID_ARG, "%s: chunk=%d not a positive multiple of 64", fn,
                          chunk);
-    if (n_kv < T)
-        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_kv=%lld < T=%d", fn, (long long)n_kv, T);
+    if (min_keys < 0)
+        min_keys = T;
+    if (n_kv < min_keys)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n_kv=%lld < %lld", fn, (long long)n_kv,
+                         (long long)min_keys);
     for (int l = 0; l < n_layers; ++l)
         if (n_kv > layers[l].capacity)
             return set_error(KVQ_ERR_INVALID_ARG, "%s: n_kv=%lld > capacity of layer %d", fn,
@@ -184,6 +188,7 @@ static kvq_status fill_decode(const kvq_layer *layers, int n_layers, const uint1
     a.q = reinterpret_cast<const __half *>(q);
     a.out_part = out_part;
     a.lse_part = lse_part;
+    a.vis_last = n_kv - T;
     KVQ_TRY(status_word(&a.status));
     // test hooks (kvq_test_set_hooks): the general kernel, a forced wait timeout
     a.force_simple = test_hooks().decode_general.load(std::memory_order_relaxed);
@@ -297,12 +302,44 @@ kvq_status kvq_decode_attn(const kvq_layer *layers, int n_layers, const uint16_t
                           lse_part, as_stream(stream));
 }
 
+kvq_status kvq_decode_attn_shard(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                                 int n_q_heads, int T, int64_t n_keys, int64_t key0,
+                                 int64_t n_kv, int chunk, float scale, float *out_part,
+                                 float *lse_part, kvq_stream stream)
+{
+    const char *fn = "kvq_decode_attn_shard";
+    KVQ_TRY(validate_decode(layers, n_layers, q, n_q_heads, T, n_keys, chunk, scale, out_part,
+                            lse_part, fn, 1));
+    if (key0 < 0 || n_kv < T || key0 > n_kv - n_keys)
+        return set_error(KVQ_ERR_INVALID_ARG,
+                         "%s: keys [%lld, %lld) not inside a context of n_kv=%lld >= T=%d", fn,
+                         (long long)key0, (long long)(key0 + n_keys), (long long)n_kv, T);
+    DecodeArgs a;
+    KVQ_TRY(fill_decode(layers, n_layers, q, n_q_heads, T, n_keys, chunk, scale, out_part,
+                        lse_part, a));
+    a.vis_last = n_kv - T - key0;  // token t sees global keys <= n_kv - T + t
+    if (!launch_decode(a, as_stream(stream)))
+        return set_error(KVQ_ERR_UNSUPPORTED, "%s: no kernel for this shape", fn);
+    return check_launch(fn);
+}
+
 kvq_status kvq_merge_lse(const float *out_part, const float *lse_part, int64_t rows,
                          int n_chunks, int head_dim, float *out, float *lse, kvq_stream stream)
 {
     const char *fn = "kvq_merge_lse";
     KVQ_TRY(validate_merge(out_part, lse_part, rows, n_chunks, head_dim, out, lse, fn));
     launch_merge_lse(out_part, lse_part, rows, n_chunks, head_dim, out, lse, as_stream(stream));
+    return check_launch(fn);
+}
+
+kvq_status kvq_merge_lse_parts(const float *out_parts, const float *lse_parts, int n_parts,
+                               int64_t rows, int head_dim, float *out, float *lse,
+                               kvq_stream stream)
+{
+    const char *fn = "kvq_merge_lse_parts";
+    KVQ_TRY(validate_merge(out_parts, lse_parts, rows, n_parts, head_dim, out, lse, fn));
+    launch_merge_lse_parts(out_parts, lse_parts, n_parts, rows, head_dim, out, lse,
+                           as_stream(stream));
     return check_launch(fn);
 }
 

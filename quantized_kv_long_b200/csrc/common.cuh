@@ -112,12 +112,17 @@ void launch_append(const MutLayerTable &t, int n_layers, int n_kv_heads, int hea
                    int n_tok, cudaStream_t s);
 void launch_merge_lse(const float *out_part, const float *lse_part, int64_t rows, int n_chunks,
                       int head_dim, float *out, float *lse, cudaStream_t s);
+void launch_merge_lse_parts(const float *out_parts, const float *lse_parts, int n_parts,
+                            int64_t rows, int head_dim, float *out, float *lse, cudaStream_t s);
 
 struct DecodeArgs {
     LayerTable layers;
     int n_layers, n_kv_heads, head_dim, n_q_heads, T;
     int k_type, v_type;  // resolved block formats (KVQ_TYPE_Q8_0 / KVQ_TYPE_Q4_0)
     int64_t n_kv;
+    // causal visibility: the row of token t sees the keys (rows of the layers) j <=
+    // vis_last + t; n_kv - T for a whole context, less for a shard of one
+    int64_t vis_last;
     int chunk;
     float scale;
     const __half *q;
@@ -128,6 +133,19 @@ struct DecodeArgs {
 };
 // Returns false (and launches nothing) if no kernel supports the shape.
 bool launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+// Argument checks and the decode launch shared by the C ABI's decode entry points
+// (api.cu).  validate_decode: n_kv must be at least min_keys (T when negative).
+kvq_status validate_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                           int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                           const float *out_part, const float *lse_part, const char *fn,
+                           int64_t min_keys = -1);
+kvq_status enqueue_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
+                          int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                          float *out_part, float *lse_part, cudaStream_t s);
+kvq_status validate_merge(const float *out_part, const float *lse_part, int64_t rows,
+                          int n_chunks, int head_dim, const float *out, const float *lse,
+                          const char *fn);
 // True for the shapes of the persistent tensor-core kernel.
 bool decode_tc_supported(const DecodeArgs &a);
 

@@ -12,7 +12,8 @@
 // page: paged decode attention over the verify batch; "Known Issues Fixed" of
 // the OSCAR2 page: the max covers complete scores; GQA section of the KV-cache
 // guide): row r = t*G + g is query head h*G + g of token t and sees keys
-// j <= n_kv - T + t of chunk c = keys [c*chunk, (c+1)*chunk).
+// j <= vis_last + t (n_kv - T + t for a whole context) of chunk c = keys
+// [c*chunk, (c+1)*chunk).
 //
 // K and V may each be in either block format (template parameters KT, VT:
 // KVQ_TYPE_Q8_0 or KVQ_TYPE_Q4_0); the pages' configuration is Q8_0 K / Q4_0 V.
@@ -66,7 +67,7 @@ decode_simple_kernel(DecodeArgs a)
             const int64_t j = j0 + jj;
             const int t = r / G;
             float s = -INFINITY;
-            if (j < c1 && j <= a.n_kv - a.T + t) {
+            if (j < c1 && j <= a.vis_last + t) {
                 const uint8_t *kr = kb + j * krow;
                 const float *qr = q_s + r * D;
                 float tot = 0.0f;

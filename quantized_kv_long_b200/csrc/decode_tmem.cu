@@ -87,7 +87,7 @@ constexpr int W_CONV = 4, W_SOFT = 12, W_VAL = 20;
 constexpr int N_CONV = 8, N_SOFT = 8, N_VAL = 8;
 constexpr int WARPS = 28, THREADS = 32 * WARPS;
 constexpr int BAR_SOFT = 1;                  // named barrier of the softmax warps
-constexpr int REG_CTL = 56, REG_CONV = 56, REG_SOFT = 88, REG_VAL = 80;  // registers per thread
+constexpr int REG_CTL = 64, REG_CONV = 56, REG_SOFT = 80, REG_VAL = 80;  // registers per thread
 static_assert(128 * (REG_CTL + 2 * REG_CONV + 2 * REG_SOFT + 2 * REG_VAL) <= THREADS * 72,
               "register split within the launch's 72 per thread");
 
@@ -581,7 +581,6 @@ __device__ __forceinline__ void role_soft(const DecodeArgs &a)
     // pair p of S buffer sb: this warp's rows of block 2p at columns [2 RH rh, +RH),
     // of block 2p+1 at [2 RH rh + RH, +RH)
     const uint32_t taddr = tbase + ((uint32_t)(32 * quad) << 16) + CF::COL_S + 2 * RH * rh;
-    const int64_t vis_last = a.n_kv - a.T;  // token t sees keys <= vis_last + t
     float m[RH], l[RH];
     bool aborted = false;
     int it = 0, ui = 0;
@@ -640,9 +639,10 @@ __device__ __forceinline__ void role_soft(const DecodeArgs &a)
             //      padded rows
             const int j = i * TOK + key;  // key index in the chunk
             const bool edge = (i + 1) * TOK > un.n_tok ||
-                              un.c0 + (int64_t)(i + 1) * TOK - 1 > vis_last || R < NR;
+                              un.c0 + (int64_t)(i + 1) * TOK - 1 > a.vis_last || R < NR;
             if (aborted || edge) {
-                const int64_t kk = un.c0 + j - vis_last;  // visible to token t iff kk <= t
+                // token t sees keys <= vis_last + t: visible iff kk <= t
+                const int64_t kk = un.c0 + j - a.vis_last;
 #pragma unroll
                 for (int r = 0; r < RH; ++r) {
                     const int rr = r0 + r;

@@ -9,9 +9,8 @@
 //
 // The order of every floating-point operation is fixed by the 64-thread group
 // (strided partial sums, a warp shuffle tree, then the two warp results added
-// in order) and by explicit fused multiply-adds, so the merge kernel (one
-// 64-thread CTA per row) and the fused decode step (64-thread groups of the
-// last CTA of a KV head) produce bit-identical rows.
+// in order) and by explicit fused multiply-adds, so a row's result does not
+// depend on the launch shape or on where its partials are stored.
 #pragma once
 
 #include "common.cuh"
@@ -46,22 +45,21 @@ __device__ __forceinline__ float group_sum(float v, float *red, int t, Sync sync
     return red[0] + red[1];
 }
 
-// Merge row partials op[c][0..head_dim) (row-major, c < n_chunks) and lp[c]
-// into o[0..head_dim) and *lse_out.  t = thread index in the group (0..63);
+// Merge row partials op[c * op_stride + 0..head_dim) and lp[c * lp_stride]
+// (c < n_chunks) into o[0..head_dim) and *lse_out.  t = thread index in the group (0..63);
 // red = 2 floats of shared memory private to the group; w_s = n_chunks floats
 // of shared memory private to the group, or nullptr (the weights are then
-// recomputed per element, with the same arithmetic).  CG: read the partials
-// through L2 only (they were written by other CTAs of the same launch).
-// head_dim % 4 == 0, op and o 16-byte aligned.
-template <bool CG, class Sync>
-__device__ __forceinline__ void merge_row(const float *op, const float *lp, int n_chunks,
-                                          int head_dim, float *o, float *lse_out, float *w_s,
-                                          float *red, int t, Sync sync)
+// recomputed per element, with the same arithmetic).
+// head_dim % 4 == 0; op, op_stride * 4 bytes and o 16-byte aligned.
+template <class Sync>
+__device__ __forceinline__ void merge_row(const float *op, int64_t op_stride, const float *lp,
+                                          int64_t lp_stride, int n_chunks, int head_dim, float *o,
+                                          float *lse_out, float *w_s, float *red, int t, Sync sync)
 {
-    auto ld = [](const float *p) -> float { return CG ? __ldcg(p) : *p; };
+    auto ld = [](const float *p) -> float { return *p; };
     float m = -INFINITY;
     for (int c = t; c < n_chunks; c += MERGE_GROUP)
-        m = fmaxf(m, ld(lp + c));
+        m = fmaxf(m, ld(lp + c * lp_stride));
     m = group_max(m, red, t, sync);
     if (m == -INFINITY) {
         for (int i = t; i < head_dim; i += MERGE_GROUP)
@@ -73,7 +71,7 @@ __device__ __forceinline__ void merge_row(const float *op, const float *lp, int 
     }
     float s = 0.0f;
     for (int c = t; c < n_chunks; c += MERGE_GROUP) {
-        const float l = ld(lp + c);
+        const float l = ld(lp + c * lp_stride);
         if (l != -INFINITY)
             s += expf(l - m);
     }
@@ -81,7 +79,7 @@ __device__ __forceinline__ void merge_row(const float *op, const float *lp, int 
     const float L = m + logf(s);
     if (w_s) {
         for (int c = t; c < n_chunks; c += MERGE_GROUP) {
-            const float l = ld(lp + c);
+            const float l = ld(lp + c * lp_stride);
             w_s[c] = (l == -INFINITY) ? 0.0f : expf(l - L);
         }
         sync();
@@ -102,14 +100,14 @@ __device__ __forceinline__ void merge_row(const float *op, const float *lp, int 
                     if (w_s) {
                         w[k] = w_s[c];
                     } else {
-                        const float l = ld(lp + c);
+                        const float l = ld(lp + c * lp_stride);
                         w[k] = (l == -INFINITY) ? 0.0f : expf(l - L);
                     }
                 }
                 if (w[k] != 0.0f) {
                     const float4 *src =
-                        reinterpret_cast<const float4 *>(op + (int64_t)c * head_dim + i);
-                    v[k] = CG ? __ldcg(src) : *src;
+                        reinterpret_cast<const float4 *>(op + (int64_t)c * op_stride + i);
+                    v[k] = *src;
                 }
             }
 #pragma unroll

@@ -31,15 +31,6 @@
 #include "common.cuh"
 
 namespace kvq {
-kvq_status validate_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
-                           int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
-                           const float *out_part, const float *lse_part, const char *fn);
-kvq_status enqueue_decode(const kvq_layer *layers, int n_layers, const uint16_t *q,
-                          int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
-                          float *out_part, float *lse_part, cudaStream_t s);
-kvq_status validate_merge(const float *out_part, const float *lse_part, int64_t rows,
-                          int n_chunks, int head_dim, const float *out, const float *lse,
-                          const char *fn);
 
 namespace {
 

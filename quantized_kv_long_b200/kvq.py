@@ -78,6 +78,9 @@ _SIGS = {
     "kvq_append": ([_LP, _I32, _P, _P, _I64, _I32, _P], _I32),
     "kvq_decode_attn": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P], _I32),
     "kvq_merge_lse": ([_P, _P, _I64, _I32, _I32, _P, _P, _P], _I32),
+    "kvq_decode_attn_shard": ([_LP, _I32, _P, _I32, _I32, _I64, _I64, _I64, _I32, _F32, _P, _P,
+                               _P], _I32),
+    "kvq_merge_lse_parts": ([_P, _P, _I32, _I64, _I32, _P, _P, _P], _I32),
     "kvq_decode_step": ([_LP, _I32, _P, _P, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P,
                          _SZ, _P], _I32),
     "kvq_prefill_attn": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P, _SZ,
@@ -173,6 +176,21 @@ def kvq_merge_lse(out_part, lse_part, rows: int, n_chunks: int, head_dim: int, o
                   stream=None) -> None:
     _check(_lib.kvq_merge_lse(_ptr(out_part), _ptr(lse_part), rows, n_chunks, head_dim,
                               _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def kvq_decode_attn_shard(layers, q, n_q_heads: int, T: int, n_keys: int, key0: int, n_kv: int,
+                          chunk: int, scale: float, out_part, lse_part, stream=None) -> None:
+    """Decode over keys [key0, key0 + n_keys) of an n_kv-key context (see include/kvq.h)."""
+    arr, n = _layers(layers)
+    _check(_lib.kvq_decode_attn_shard(arr, n, _ptr(q), n_q_heads, T, n_keys, key0, n_kv, chunk,
+                                      scale, _ptr(out_part), _ptr(lse_part), _stream(stream)))
+
+
+def kvq_merge_lse_parts(out_parts, lse_parts, n_parts: int, rows: int, head_dim: int, out, lse,
+                        stream=None) -> None:
+    """Merge part-major partials [n_parts][rows][head_dim] (see include/kvq.h)."""
+    _check(_lib.kvq_merge_lse_parts(_ptr(out_parts), _ptr(lse_parts), n_parts, rows, head_dim,
+                                    _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def kvq_decode_step(layers, k_new, v_new, q, n_q_heads: int, T: int, n_kv: int, chunk: int,
