@@ -95,12 +95,10 @@ typedef void *kvq_stream;
 /* One attention layer of the cache.  All layers passed to one call must have
  * the same n_kv_heads and head_dim. */
 /* Block format of a cache tensor.  KVQ_TYPE_DEFAULT is Q8_0 for K and Q4_0
- * for V.  All layers passed to one call must use the same formats.  Append,
- * the general decode path (kvq_decode_attn, kvq_decode_step,
- * kvq_decode_merged_static, kvq_stream_decode) accept every combination; the
- * tiled decode kernels, the fused step's single launch and kvq_prefill_attn
- * implement the default pair only (decode falls back to the general kernel,
- * the step to three launches, prefill returns KVQ_ERR_UNSUPPORTED). */
+ * for V.  All layers passed to one call must use the same formats.  Every call
+ * accepts every combination; the tensor-core kernels are built for the
+ * default pair (decode and prefill run the other pairs on their general,
+ * CUDA-core kernels). */
 typedef enum kvq_type {
     KVQ_TYPE_DEFAULT = 0,
     KVQ_TYPE_Q8_0 = 1,   /* 34 B per 32 elements */

@@ -5,8 +5,8 @@
 // keys processed in tiles of 64 with an online softmax.  K and V are read
 // from global memory and dequantized in registers; the per-block K scale is
 // applied to each block's fp32 partial dot product, so only fp32 rounding
-// separates it from the exact result.  It serves the shapes the tiled tensor-
-// core kernel (decode.cu) does not cover, and is the correctness baseline.
+// separates it from the exact result.  It serves the shapes and formats the
+// persistent tensor-core kernel (decode_tmem.cu) does not cover.
 //
 // Semantics (speculative-decoding paragraph of the RX 9070 XT KV-streaming
 // page: paged decode attention over the verify batch; "Known Issues Fixed" of

@@ -9,11 +9,12 @@
 // online (running max, running sum) merge carried across pages of keys
 // inside the kernel.
 //
-// Two kernels:
+// Kernels:
 //  * prefill_tc_kernel -- the tensor-core path (tcgen05, TMEM) for rows that
-//    see at least PF_MIN_KEYS keys.  One CTA per (128 query rows of one KV
-//    head's group, KV head, layer); rows are (token, q head) pairs.  Per tile
-//    of 32 keys:
+//    see at least PF_MIN_KEYS keys (Q8_0 K / Q4_0 V at head_dim 256).  One CTA
+//    per (128 query rows of one KV head's group, (layer, KV head) pair); rows
+//    are (token, q head) pairs.  Per tile of 32 keys, in the variant that
+//    dequantizes in the CTA (PRE = false):
 //      - a producer thread bulk-copies the tile's raw Q8_0 K head-rows (32 x
 //        272 B) and Q4_0 V head-rows (32 x 144 B) into a 4-slot staging ring,
 //        so that three tiles of copies are in flight while one is dequantized;
@@ -35,6 +36,13 @@
 //        read S, apply the causal mask, keep a lazy running max (moves only
 //        when a score exceeds it by 8 in log2 units, with an exact rescale of
 //        O in TMEM) and write P = 2^(s - m) as f16 back into the slot.
+//    With a workspace (PRE = true) prefill_expand_kernel first writes every
+//    tile of a (layer, KV head) pair once as its three swizzled f16 images into
+//    the pair's slab; the tensor-core kernel then bulk-copies the images into 4
+//    slots (no dequant warps) and runs 8 softmax warps, two per TMEM lane
+//    quadrant, each owning 16 of a tile's keys.  A workspace of fewer slabs than
+//    pairs is used in chunks of pairs through its two halves, alternating
+//    between the caller's stream and a second one (launch_prefill).
 //    V^ and P carry one f16 rounding each (relative 2^-11).  These errors are
 //    independent per key and average over the visible keys, but a row whose
 //    softmax is peaked (a large query component on an x8 outlier channel) can
@@ -46,8 +54,11 @@
 //    8.8e-5 at 262,144 (tolerance 2e-3).  Rows that see fewer than
 //    PF_MIN_KEYS = 16,384 keys take the exact kernel.
 //  * prefill_exact_kernel -- CUDA cores, fp32 with per-block scaling (the
-//    same arithmetic as the general decode kernel), for rows that see fewer
-//    than PF_MIN_KEYS keys.
+//    same arithmetic as the general decode kernel), templated on both block
+//    formats, for rows that see fewer than PF_MIN_KEYS keys, for every other
+//    format pair and head_dim, and for calls that ask for per-page partials
+//    (a page is a short context, where the f16 rounding above misses the
+//    tolerance: measured 4.0-5.2e-3).
 // Every mbarrier wait is bounded; a wait that runs out records
 // KVQ_ERR_TIMEOUT in the status word and the roles fall through, waiting
 // (bounded) for their own copies and MMAs before the CTA frees TMEM and exits.

@@ -1,6 +1,6 @@
 // quant.cuh -- one warp quantizes one 32-element block (Q8_0 or Q4_0).
 //
-// Used by the append and quantize kernels and by the fused decode step.  Every
+// Used by the append and quantize kernels.  Every
 // arithmetic step is an explicitly rounded fp32 operation (__fdiv_rn,
 // __fmul_rn, __fadd_rn), so the blocks do not depend on the compiler's
 // multiply-add contraction and are bit-identical wherever these run.
