@@ -39,10 +39,9 @@
 //    With a workspace (PRE = true) prefill_expand_kernel first writes every
 //    tile of a (layer, KV head) pair once as its three swizzled f16 images into
 //    the pair's slab; the tensor-core kernel then bulk-copies the images into 4
-//    slots (no dequant warps) and runs 8 softmax warps, two per TMEM lane
-//    quadrant, each owning 16 of a tile's keys.  A workspace of fewer slabs than
-//    pairs is used in chunks of pairs through its two halves, alternating
-//    between the caller's stream and a second one (launch_prefill).
+//    slots (no dequant warps).  A workspace of fewer slabs than pairs is used in
+//    chunks of pairs through its two halves, alternating between the caller's
+//    stream and a second one (launch_prefill).
 //    V^ and P carry one f16 rounding each (relative 2^-11).  These errors are
 //    independent per key and average over the visible keys, but a row whose
 //    softmax is peaked (a large query component on an x8 outlier channel) can
@@ -86,9 +85,10 @@ constexpr int N_SOFT = 4, N_DEQ = 8;
 // roles: softmax warps, dequant warps (none when the f16 tiles were expanded into
 // the workspace beforehand), the producer warp, the MMA warp
 template <bool PRE> constexpr int n_deq() { return PRE ? 0 : N_DEQ; }
-// softmax warps: one per TMEM lane quadrant, or two (each with half of a tile's keys)
-// when no dequant warps compete for the issue slots
-template <bool PRE> constexpr int n_soft() { return PRE ? 2 * N_SOFT : N_SOFT; }
+// softmax warps: one per TMEM lane quadrant, each with all 32 keys of a tile (P
+// overwrites the tile's scores in tensor memory, so a warp that shared a quadrant
+// would need a per-tile barrier before writing it; measured slower)
+template <bool PRE> constexpr int n_soft() { return N_SOFT; }
 template <bool PRE> constexpr int w_prod() { return n_soft<PRE>() + n_deq<PRE>(); }
 template <bool PRE> constexpr int w_mma() { return w_prod<PRE>() + 1; }
 template <bool PRE> constexpr int pf_threads() { return (w_mma<PRE>() + 1) * 32; }  // 14 / 6 warps
@@ -118,8 +118,6 @@ struct PfSmemHead {
         pv_done[NS], q_ready;
     uint64_t mma_drain;              // one commit after the last MMA: all of them are done
     uint64_t never;                  // test hook: a barrier that nothing completes
-    uint64_t xch[N_SOFT];            // two softmax warps per quadrant: the final sums
-    float xmx[2][2][BM];             // [warp half][phase parity][row]: tile max, then l
     uint32_t tmem_base;
     int abort;
 };
@@ -321,8 +319,6 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         ptx::mbar_init(&hd.q_ready, n_soft<PRE>());
         ptx::mbar_init(&hd.mma_drain, 1);
         ptx::mbar_init(&hd.never, 1);
-        for (int i = 0; i < N_SOFT; ++i)
-            ptx::mbar_init(&hd.xch[i], 2);
         hd.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -351,34 +347,22 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
 
     if (warp < n_soft<PRE>()) {
         // ================================================================ softmax
-        // Warp (quad, hf) owns the query rows of TMEM lane quadrant quad (one row per
-        // thread).  With NH = 2 warps per quadrant, warp hf takes keys [16 hf, 16 hf + 16)
-        // of every tile and columns [128 hf, 128 hf + 128) of O; the pair agrees on the
-        // running max through hd.xch / hd.xmx once per tile.  The arithmetic does not
-        // depend on NH: each 16-key half of a tile has its own running sum l[hh],
-        // l = l[0] + l[1] at the end, and the max is exact.
-        constexpr int NH = n_soft<PRE>() / N_SOFT;
-        const int quad = warp & 3, hf = warp >> 2;
-        const int h0 = NH == 2 ? hf : 0;  // this warp's halves: [h0, h0 + 2 / NH)
+        // Warp quad owns the query rows of TMEM lane quadrant quad (one row per thread)
+        // and all 32 keys of every tile: it reads the tile's scores, then writes P over
+        // them.  Each 8-key group g of a tile has its own running sum l_g; l = (l_0 +
+        // l_1) + (l_2 + l_3) at the end.
+        const int quad = warp & 3;
         const int i = quad * 32 + lane;   // query row of this thread = its TMEM lane
         const int gr = R0 + i;
         const bool live = gr <= r_last;
         const int t = live ? gr / G : 0, gq = live ? gr % G : 0;
         const int64_t lim = a.n_cached + t;  // last visible key
         const uint32_t lane_addr = tbase + ((uint32_t)(quad * 32) << 16);
-        // bounded wait on the pair's exchange barrier (phase ph); false: give up
-        auto pair_sync = [&](uint32_t ph) -> bool {
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                ptx::mbar_arrive(&hd.xch[quad]);
-            return wwait(&hd.xch[quad], ph & 1u);
-        };
         {   // Q row -> TMEM columns [COL_Q, COL_Q + 128): two f16 per column, lower dim low
             const uint4 *qp = reinterpret_cast<const uint4 *>(
                 a.q + (((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq) * HD);
 #pragma unroll
-            for (int c = h0 * 4; c < h0 * 4 + 8 / NH; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 uint32_t r[16];
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
@@ -397,31 +381,21 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                 ptx::mbar_arrive(&hd.q_ready);
         }
         const float sl2 = a.scale * LOG2E;
-        constexpr int NHALF = 2 / NH;       // 16-key halves whose P and l this warp makes
-        float m = M_INIT, l[NHALF];         // l[k]: running sum of half h0 + k
+        float m = M_INIT, l[4];             // l[g]: running sum of 8-key group g
 #pragma unroll
-        for (int k = 0; k < NHALF; ++k)
+        for (int k = 0; k < 4; ++k)
             l[k] = 0.0f;
         const int64_t row_out = ((int64_t)layer * a.T + t) * a.n_q_heads + (int64_t)h * G + gq;
-        uint32_t xph = 0;  // phases of the pair's exchange barrier used so far
         // out = O / l and lse = (m + log2 l) ln 2 of this thread's row into dsto / dstl,
-        // once the PV of tile `last` is done; l = l[0] + l[1] (the two warps of a
-        // quadrant add their halves, half 0 first).  false: a wait ran out.
-        auto emit = [&](int last, float *dsto, float *dstl, uint32_t ph) -> bool {
-            bool done = wwait(&hd.pv_done[slot(last, NS)], par(last, NS));
-            float lt = l[0] + l[NHALF - 1];  // NH == 1: l of half 0 + l of half 1
-            if (NH == 2 && done) {
-                hd.xmx[hf][ph & 1][i] = l[0];
-                done = pair_sync(ph);
-                if (done)
-                    lt = hd.xmx[0][ph & 1][i] + hd.xmx[1][ph & 1][i];
-            }
-            if (!done)
+        // once the PV of tile `last` is done.  false: a wait ran out.
+        auto emit = [&](int last, float *dsto, float *dstl) -> bool {
+            if (!wwait(&hd.pv_done[slot(last, NS)], par(last, NS)))
                 return false;
+            const float lt = (l[0] + l[1]) + (l[2] + l[3]);
             ptx::tc_fence_after();
             const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
             float4 *op = reinterpret_cast<float4 *>(dsto);
-            for (int c = h0 * 8; c < h0 * 8 + 16 / NH; ++c) {
+            for (int c = 0; c < 16; ++c) {
                 uint32_t r[16];
                 ptx::tmem_ld16(lane_addr + COL_O + 16 * c, r);
                 ptx::tmem_wait_ld();
@@ -434,7 +408,7 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                                                     __uint_as_float(r[4 * v + 3]) * inv);
                 }
             }
-            if (live && h0 == 0)
+            if (live)
                 *dstl = lt > 0.0f ? (m + log2f(lt)) * LN2 : -INFINITY;
             return true;
         };
@@ -447,37 +421,28 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                 break;
             }
             ptx::tc_fence_after();
-            // every warp reads the whole tile's scores, so that both warps of a quadrant
-            // take the same max without talking to each other; s[0] holds this warp's
-            // first half (h0), s[1] the other one
-            float s[2][16];
+            // every warp reads the whole tile's 32 scores (keys in order)
+            float sc[BN];
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 uint32_t r[16];
-                ptx::tmem_ld16(lane_addr + scol + 16 * (k == 0 ? h0 : 1 - h0), r);
+                ptx::tmem_ld16(lane_addr + scol + 16 * k, r);
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    s[k][e] = __uint_as_float(r[e]);
+                    sc[16 * k + e] = __uint_as_float(r[e]);
             }
             ptx::tmem_wait_ld();
             const int64_t kj0 = (int64_t)j * BN;
             if (kj0 + BN - 1 > lim) {  // causal edge / end of the keys
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int64_t kb0 = kj0 + 16 * (k == 0 ? h0 : 1 - h0);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (kb0 + e > lim)
-                            s[k][e] = -INFINITY;
-                }
+                for (int e = 0; e < BN; ++e)
+                    if (kj0 + e > lim)
+                        sc[e] = -INFINITY;
             }
             float mx8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                mx8[e] = fmaxf(s[0][e], s[0][e + 8]);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                mx8[e & 7] = fmaxf(mx8[e & 7], s[1][e]);
+                mx8[e] = fmaxf(fmaxf(sc[e], sc[e + 8]), fmaxf(sc[e + 16], sc[e + 24]));
             // scaling is monotonic: the max of the scaled scores
             const float mx = sl2 * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
@@ -486,7 +451,7 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                 alpha = ptx::ex2(m - mx);
                 m = mx;
 #pragma unroll
-                for (int k = 0; k < NHALF; ++k)
+                for (int k = 0; k < 4; ++k)
                     l[k] *= alpha;
             }
             // rescale this warp's columns of O (rare): the whole warp takes part once any
@@ -497,7 +462,7 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                     break;
                 }
                 ptx::tc_fence_after();
-                for (int c = h0 * 8; c < h0 * 8 + 16 / NH; ++c) {
+                for (int c = 0; c < 16; ++c) {
                     uint32_t r[16];
                     ptx::tmem_ld16(lane_addr + COL_O + 16 * c, r);
                     ptx::tmem_wait_ld();
@@ -508,23 +473,23 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
                 }
                 ptx::tmem_wait_st();
             }
-            // P = 2^(s scale - m) in f16 (keys 2e, 2e + 1 of half hh in column 8 hh + e of
-            // this S slot), and the half's sum
+            // P = 2^(s scale - m) in f16 (keys 2e, 2e + 1 of the tile in column e of this S
+            // slot), and each 8-key group's sum ((p0 + p1) + (p2 + p3)) + ((p4 + p5) +
+            // (p6 + p7))
+            uint32_t pk[16];
 #pragma unroll
-            for (int k = 0; k < NHALF; ++k) {
-                const float *sh = s[k];  // half h0 + k
-                uint32_t pk[8];
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int k = 0; k < 4; ++k) {
+                float pr[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float p0 = ptx::ex2(fmaf(sh[2 * e], sl2, -m));
-                    const float p1 = ptx::ex2(fmaf(sh[2 * e + 1], sl2, -m));
-                    ls[e & 3] += p0 + p1;
-                    pk[e] = ptx::h2_bits(__floats2half2_rn(p0, p1));
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = ptx::ex2(fmaf(sc[8 * k + 2 * e], sl2, -m));
+                    const float p1 = ptx::ex2(fmaf(sc[8 * k + 2 * e + 1], sl2, -m));
+                    pr[e] = p0 + p1;
+                    pk[4 * k + e] = ptx::h2_bits(__floats2half2_rn(p0, p1));
                 }
-                l[k] += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                ptx::tmem_st8(lane_addr + scol + 8 * (h0 + k), pk);
+                l[k] += (pr[0] + pr[1]) + (pr[2] + pr[3]);
             }
+            ptx::tmem_st16(lane_addr + scol, pk);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -534,7 +499,7 @@ __global__ void __launch_bounds__(pf_threads<PRE>(), 1) prefill_tc_kernel(const 
         if (!ok && lane == 0)
             fail();
         // ---- epilogue: out = O / l, lse = (m + log2 l) ln 2, l = l[0] + l[1]
-        if (ok && !*abort && !emit(ntiles - 1, a.out + row_out * HD, a.lse + row_out, xph++) &&
+        if (ok && !*abort && !emit(ntiles - 1, a.out + row_out * HD, a.lse + row_out) &&
             lane == 0)
             fail();
     } else if (warp < W_PROD) {
