@@ -10,10 +10,11 @@ the header of ``kvq_oracle.c``.
 Every function here takes and returns numpy arrays.  Caches use the layout of
 one layer: K ``[n_kv_heads, capacity, head_dim // 32 * 34]`` uint8 and V
 ``[n_kv_heads, capacity, head_dim // 32 * 18]`` uint8 in the main (Q8_0 K /
-Q4_0 V) configuration; either tensor may use the other block format
-(``empty_cache(..., k_fmt=, v_fmt=)``), and the functions read each tensor's
-format from its head-row length (34 or 18 bytes per 32 elements, never both
-for head_dim <= 512).
+Q4_0 V) configuration; either tensor may use another block format
+(``empty_cache(..., k_fmt=, v_fmt=)``: Q8_0, Q4_0 or the INT2 OSCAR2 block of
+36 bytes per 128 elements), and the functions read each tensor's format from
+its head-row length and the head_dim of their other inputs (at a given
+head_dim the three formats give three different row lengths).
 
 Parity pins: every function below is pinned by the CPU tests (golden blocks,
 closed forms, library cross-checks, invariants); none is "parity unpinned".
@@ -30,8 +31,11 @@ from .build import build_oracle, library_path
 QK = 32
 Q8_0_BYTES = 34
 Q4_0_BYTES = 18
-FMT_Q8_0, FMT_Q4_0 = 1, 2
-_BLOCK_BYTES = {FMT_Q8_0: Q8_0_BYTES, FMT_Q4_0: Q4_0_BYTES}
+QK_OSCAR2 = 128
+OSCAR2_BYTES = 36
+FMT_Q8_0, FMT_Q4_0, FMT_OSCAR2 = 1, 2, 3
+_BLOCK_BYTES = {FMT_Q8_0: Q8_0_BYTES, FMT_Q4_0: Q4_0_BYTES, FMT_OSCAR2: OSCAR2_BYTES}
+_BLOCK_ELEMS = {FMT_Q8_0: QK, FMT_Q4_0: QK, FMT_OSCAR2: QK_OSCAR2}
 
 _lib = None
 
@@ -55,6 +59,8 @@ def _load():
         "orc_quantize_q4_0": ([P, P, i64], None),
         "orc_dequant_q8_0": ([P, P, i64], None),
         "orc_dequant_q4_0": ([P, P, i64], None),
+        "orc_quantize_oscar2": ([P, P, i64], None),
+        "orc_dequant_oscar2": ([P, P, i64], None),
         "orc_append": ([P, P, i32, i32, i64, P, P, i64, i64, i32, i32], None),
         "orc_decode_attn": ([P, P, i32, i32, i64, P, i32, i32, i64, i64, f64, P, P, i32, i32],
                             None),
@@ -102,11 +108,11 @@ def f16_bits_to_f64(h: np.ndarray) -> np.ndarray:
 
 # ---- quantizers -------------------------------------------------------------
 
-def _quant(fn, nbytes, x):
+def _quant(fn, nbytes, x, elems=QK):
     x = np.ascontiguousarray(x, dtype=np.float32)
-    if x.size % QK:
-        raise ValueError("element count must be a multiple of 32")
-    out = np.empty(x.size // QK * nbytes, dtype=np.uint8)
+    if x.size % elems:
+        raise ValueError(f"element count must be a multiple of {elems}")
+    out = np.empty(x.size // elems * nbytes, dtype=np.uint8)
     fn(_ptr(x), _ptr(out), x.size)
     return out
 
@@ -121,11 +127,16 @@ def quantize_q4_0(x: np.ndarray) -> np.ndarray:
     return _quant(_load().orc_quantize_q4_0, Q4_0_BYTES, x)
 
 
-def _dequant(fn, nbytes, b):
+def quantize_oscar2(x: np.ndarray) -> np.ndarray:
+    """OSCAR2 INT2 blocks (36 B per 128 elements) of ``x`` in memory order."""
+    return _quant(_load().orc_quantize_oscar2, OSCAR2_BYTES, x, QK_OSCAR2)
+
+
+def _dequant(fn, nbytes, b, elems=QK):
     b = np.ascontiguousarray(b, dtype=np.uint8).reshape(-1)
     if b.size % nbytes:
         raise ValueError("byte count must be a multiple of the block size")
-    out = np.empty(b.size // nbytes * QK, dtype=np.float64)
+    out = np.empty(b.size // nbytes * elems, dtype=np.float64)
     fn(_ptr(b), _ptr(out), out.size)
     return out
 
@@ -138,43 +149,52 @@ def dequant_q4_0(b: np.ndarray) -> np.ndarray:
     return _dequant(_load().orc_dequant_q4_0, Q4_0_BYTES, b)
 
 
+def dequant_oscar2(b: np.ndarray) -> np.ndarray:
+    return _dequant(_load().orc_dequant_oscar2, OSCAR2_BYTES, b, QK_OSCAR2)
+
+
 # ---- cache ------------------------------------------------------------------
 
 def empty_cache(n_kv_heads: int, head_dim: int, capacity: int, k_fmt: int = FMT_Q8_0,
                 v_fmt: int = FMT_Q4_0):
     """Zeroed K and V byte arrays of one layer (K blocks in ``k_fmt``, V in ``v_fmt``)."""
-    k = np.zeros((n_kv_heads, capacity, head_dim // QK * _BLOCK_BYTES[k_fmt]), dtype=np.uint8)
-    v = np.zeros((n_kv_heads, capacity, head_dim // QK * _BLOCK_BYTES[v_fmt]), dtype=np.uint8)
+    for f in (k_fmt, v_fmt):
+        if head_dim % _BLOCK_ELEMS[f]:
+            raise ValueError(f"head_dim {head_dim} is not a multiple of the block size")
+    k = np.zeros((n_kv_heads, capacity, head_dim // _BLOCK_ELEMS[k_fmt] * _BLOCK_BYTES[k_fmt]),
+                 dtype=np.uint8)
+    v = np.zeros((n_kv_heads, capacity, head_dim // _BLOCK_ELEMS[v_fmt] * _BLOCK_BYTES[v_fmt]),
+                 dtype=np.uint8)
     return k, v
 
 
-def _fmt_dim(row_bytes: int) -> tuple[int, int]:
-    """(block format, head_dim) of a head-row of ``row_bytes``: exactly one of the two
-    formats fits when head_dim <= 512."""
-    fits = [(f, row_bytes // b * QK) for f, b in _BLOCK_BYTES.items()
-            if row_bytes % b == 0 and row_bytes // b * QK <= 512]
-    assert len(fits) == 1, f"head-row of {row_bytes} bytes"
+def _fmt_of(row_bytes: int, head_dim: int) -> int:
+    """Block format of a head-row of ``row_bytes`` at ``head_dim``: at one head_dim the
+    formats' row lengths (34, 18 and 9 bytes per 32 elements) all differ."""
+    fits = [f for f in _BLOCK_BYTES
+            if head_dim % _BLOCK_ELEMS[f] == 0
+            and head_dim // _BLOCK_ELEMS[f] * _BLOCK_BYTES[f] == row_bytes]
+    if len(fits) != 1:
+        raise ValueError(f"no block format has {row_bytes}-byte head-rows at head_dim {head_dim}")
     return fits[0]
 
 
-def _cache_dims(k_cache, v_cache):
-    """(n_kv_heads, head_dim, capacity, k_fmt, v_fmt) of one layer's caches."""
+def _cache_dims(k_cache, v_cache, head_dim: int):
+    """(n_kv_heads, capacity, k_fmt, v_fmt) of one layer's caches read at ``head_dim``."""
     H, cap, kb = k_cache.shape
-    k_fmt, D = _fmt_dim(kb)
-    v_fmt, Dv = _fmt_dim(v_cache.shape[2])
-    assert v_cache.shape[:2] == (H, cap) and Dv == D
+    assert v_cache.shape[:2] == (H, cap)
     assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
-    return H, D, cap, k_fmt, v_fmt
+    return H, cap, _fmt_of(kb, head_dim), _fmt_of(v_cache.shape[2], head_dim)
 
 
 def append(k_cache, v_cache, k_new, v_new, pos: int) -> None:
     """Quantize rows ``k_new``/``v_new`` ``[n_tok, n_kv_heads, head_dim]`` into rows
     ``[pos, pos + n_tok)`` of the caches, in place."""
-    H, D0, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache)
     k_new = np.ascontiguousarray(k_new, dtype=np.float32)
     v_new = np.ascontiguousarray(v_new, dtype=np.float32)
     n_tok, h2, D = k_new.shape
-    if h2 != H or D != D0 or v_new.shape != k_new.shape or pos < 0 or pos + n_tok > cap:
+    H, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache, D)
+    if h2 != H or v_new.shape != k_new.shape or pos < 0 or pos + n_tok > cap:
         raise ValueError("bad append shape")
     _load().orc_append(_ptr(k_cache), _ptr(v_cache), H, D, cap, _ptr(k_new), _ptr(v_new),
                        pos, n_tok, k_fmt, v_fmt)
@@ -187,10 +207,10 @@ def decode_attn(k_cache, v_cache, q: np.ndarray, n_kv: int, chunk: int, scale: f
 
     Returns ``(out_part [T, Hq, n_chunks, D] f64, lse_part [T, Hq, n_chunks] f64)``.
     """
-    H, D, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache)
     q = np.ascontiguousarray(q, dtype=np.float16)
-    T, Hq, D2 = q.shape
-    assert D2 == D and Hq % H == 0 and 1 <= T <= n_kv <= cap and chunk >= 1
+    T, Hq, D = q.shape
+    H, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache, D)
+    assert Hq % H == 0 and 1 <= T <= n_kv <= cap and chunk >= 1
     n_chunks = -(-n_kv // chunk)
     out = np.empty((T, Hq, n_chunks, D), dtype=np.float64)
     lse = np.empty((T, Hq, n_chunks), dtype=np.float64)
@@ -215,9 +235,9 @@ def merge_lse(out_part: np.ndarray, lse_part: np.ndarray):
 def attn_rows(k_cache, v_cache, q_rows: np.ndarray, q_head: np.ndarray, n_q_heads: int,
               key_begin: np.ndarray, key_end: np.ndarray, scale: float):
     """One-pass attention of arbitrary rows (fp16 ``q_rows [n, D]``)."""
-    H, D, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache)
     q_rows = np.ascontiguousarray(q_rows, dtype=np.float16)
-    n = q_rows.shape[0]
+    n, D = q_rows.shape
+    H, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache, D)
     q_head = np.ascontiguousarray(q_head, dtype=np.int32)
     kb = np.ascontiguousarray(key_begin, dtype=np.int64)
     ke = np.ascontiguousarray(key_end, dtype=np.int64)
@@ -238,9 +258,9 @@ def prefill_attn(k_cache, v_cache, q: np.ndarray, n_cached: int, page: int, scal
     Returns ``(out [T, Hq, D], lse [T, Hq])`` and, with ``pages=True``, also
     ``(page_out [T, Hq, n_pages, D], page_lse [T, Hq, n_pages])``.
     """
-    H, D, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache)
     q = np.ascontiguousarray(q, dtype=np.float16)
-    T, Hq, _ = q.shape
+    T, Hq, D = q.shape
+    H, cap, k_fmt, v_fmt = _cache_dims(k_cache, v_cache, D)
     assert n_cached + T <= cap and Hq % H == 0
     n_pages = -(-(n_cached + T) // page)
     out = np.empty((T, Hq, D), dtype=np.float64)

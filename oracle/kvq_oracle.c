@@ -35,6 +35,16 @@
  *    the first element of largest |x|; d = m/-8; id = d ? 1/d : 0;
  *    u = min(15, trunc(x*id + 8.5)) with the product and the sum each rounded
  *    to fp32.  Dequant: d*(u-8).
+ *  - OSCAR2 block (36 B per 128 elements; [OSCAR2] Compression Ratios table:
+ *    2.25 bits per element, INT2 codes with fp16 zero-point metadata): fp16 d,
+ *    fp16 m (the zero-point: the value code 0 decodes to), then 32 bytes;
+ *    byte j holds the 2-bit codes of elements j, j+32, j+64, j+96 in bits
+ *    0-1, 2-3, 4-5, 6-7.  In fp32, no fused multiply-add: mn = min x,
+ *    mx = max x; d = (mx - mn)/3; id = d ? 1/d : 0;
+ *    u = min(3, trunc((x - mn)*id + 0.5)), each operation rounded to fp32.
+ *    fp16(d) and fp16(mn) are stored.  Dequant: d*u + m.  The page's Hadamard
+ *    rotation is baked into the model weights offline ("Rotation Model
+ *    Conversion"), so rows arrive rotated and nothing here rotates them.
  *  - fp32 -> fp16 is IEEE round-to-nearest-even with subnormals.
  *  - Attention (fp64): s_j = scale * sum_i q_i * k^_ij; m = max_j s_j;
  *    l = sum_j exp(s_j - m); o = sum_j exp(s_j - m) v^_j / l; lse = m + ln l.
@@ -49,10 +59,11 @@
  * Cache layout of one layer (the interface both sides implement):
  *   K: [n_kv_heads][capacity][head_dim/32] Q8_0 blocks (34 B each)
  *   V: [n_kv_heads][capacity][head_dim/32] Q4_0 blocks (18 B each)
- * The pages' main configuration.  Each tensor may also use the other format
+ * The pages' main configuration.  Each tensor may also use another format
  * (q8_0/q8_0 and q4_0/q4_0 caches are the other choices of the KV-cache
- * guide's levers section): the cache functions take the block format of K and
- * of V (FMT_Q8_0 or FMT_Q4_0), and a head-row is head_dim/32 blocks of it.
+ * guide's levers section; oscar2 is [OSCAR2]'s INT2 format): the cache
+ * functions take the block format of K and of V (FMT_Q8_0, FMT_Q4_0 or
+ * FMT_OSCAR2), and a head-row is head_dim / (elements per block) blocks of it.
  *
  * Build: gcc -std=c11 -O2 -fopenmp -ffp-contract=off -fPIC -shared.
  * Floating-point contraction must stay off: the quantizers are defined as a
@@ -69,8 +80,11 @@
 #define QK 32
 #define Q8_0_BYTES 34
 #define Q4_0_BYTES 18
+#define QK_OSCAR2 128
+#define OSCAR2_BYTES 36
 #define FMT_Q8_0 1
 #define FMT_Q4_0 2
+#define FMT_OSCAR2 3
 
 /* ------------------------------------------------------------------------ */
 /* fp16 <-> fp32, written from the IEEE 754 binary16 definition.            */
@@ -198,6 +212,38 @@ static void quant_block_q4_0(const float *x, uint8_t *b)
     }
 }
 
+static void quant_block_oscar2(const float *x, uint8_t *b)
+{
+    float mn = x[0], mx = x[0];
+    for (int i = 1; i < QK_OSCAR2; ++i) {
+        if (x[i] < mn)
+            mn = x[i];
+        if (x[i] > mx)
+            mx = x[i];
+    }
+    float range = mx - mn;
+    float d = range / 3.0f;
+    float id = (d != 0.0f) ? 1.0f / d : 0.0f;
+    uint16_t dh = f32_to_f16(d), mh = f32_to_f16(mn);
+    b[0] = (uint8_t)(dh & 0xff);
+    b[1] = (uint8_t)(dh >> 8);
+    b[2] = (uint8_t)(mh & 0xff);
+    b[3] = (uint8_t)(mh >> 8);
+    for (int j = 0; j < 32; ++j) {
+        int byte = 0;
+        for (int k = 0; k < 4; ++k) {
+            float diff = x[j + 32 * k] - mn;
+            float p = diff * id;
+            float s = p + 0.5f;
+            int u = (int)truncf(s);
+            if (u > 3)
+                u = 3;
+            byte |= u << (2 * k);
+        }
+        b[4 + j] = (uint8_t)byte;
+    }
+}
+
 void orc_quantize_q8_0(const float *x, uint8_t *blocks, int64_t n)
 {
     int64_t nb = n / QK;
@@ -212,6 +258,14 @@ void orc_quantize_q4_0(const float *x, uint8_t *blocks, int64_t n)
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < nb; ++i)
         quant_block_q4_0(x + i * QK, blocks + i * Q4_0_BYTES);
+}
+
+void orc_quantize_oscar2(const float *x, uint8_t *blocks, int64_t n)
+{
+    int64_t nb = n / QK_OSCAR2;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nb; ++i)
+        quant_block_oscar2(x + i * QK_OSCAR2, blocks + i * OSCAR2_BYTES);
 }
 
 /* Dequantization is exact in fp64 (and in fp32): an fp16 times a small int. */
@@ -231,6 +285,17 @@ static void dequant_block_q4_0(const uint8_t *b, double *y)
     }
 }
 
+/* d*u + m is exact in fp64: every finite fp16 is a multiple of 2^-24 below
+ * 2^16, so d*u + m is a multiple of 2^-24 below 2^18 (42 significant bits). */
+static void dequant_block_oscar2(const uint8_t *b, double *y)
+{
+    double d = f16_to_f64((uint16_t)(b[0] | (b[1] << 8)));
+    double m = f16_to_f64((uint16_t)(b[2] | (b[3] << 8)));
+    for (int j = 0; j < 32; ++j)
+        for (int k = 0; k < 4; ++k)
+            y[j + 32 * k] = d * (double)((b[4 + j] >> (2 * k)) & 3) + m;
+}
+
 void orc_dequant_q8_0(const uint8_t *blocks, double *x, int64_t n)
 {
     for (int64_t i = 0; i < n / QK; ++i)
@@ -243,28 +308,46 @@ void orc_dequant_q4_0(const uint8_t *blocks, double *x, int64_t n)
         dequant_block_q4_0(blocks + i * Q4_0_BYTES, x + i * QK);
 }
 
+void orc_dequant_oscar2(const uint8_t *blocks, double *x, int64_t n)
+{
+    for (int64_t i = 0; i < n / QK_OSCAR2; ++i)
+        dequant_block_oscar2(blocks + i * OSCAR2_BYTES, x + i * QK_OSCAR2);
+}
+
 /* ------------------------------------------------------------------------ */
-/* Cache layout helpers: a block format is FMT_Q8_0 or FMT_Q4_0             */
+/* Cache layout helpers: a block format is FMT_Q8_0, FMT_Q4_0 or FMT_OSCAR2 */
 /* ------------------------------------------------------------------------ */
 
-static size_t block_bytes(int fmt) { return fmt == FMT_Q8_0 ? Q8_0_BYTES : Q4_0_BYTES; }
+static int block_elems(int fmt) { return fmt == FMT_OSCAR2 ? QK_OSCAR2 : QK; }
 
-static size_t row_bytes(int fmt, int head_dim) { return (size_t)(head_dim / QK) * block_bytes(fmt); }
+static size_t block_bytes(int fmt)
+{
+    return fmt == FMT_Q8_0 ? Q8_0_BYTES : fmt == FMT_Q4_0 ? Q4_0_BYTES : OSCAR2_BYTES;
+}
+
+static size_t row_bytes(int fmt, int head_dim)
+{
+    return (size_t)(head_dim / block_elems(fmt)) * block_bytes(fmt);
+}
 
 static void quant_block(int fmt, const float *x, uint8_t *b)
 {
     if (fmt == FMT_Q8_0)
         quant_block_q8_0(x, b);
-    else
+    else if (fmt == FMT_Q4_0)
         quant_block_q4_0(x, b);
+    else
+        quant_block_oscar2(x, b);
 }
 
 static void dequant_block(int fmt, const uint8_t *b, double *y)
 {
     if (fmt == FMT_Q8_0)
         dequant_block_q8_0(b, y);
-    else
+    else if (fmt == FMT_Q4_0)
         dequant_block_q4_0(b, y);
+    else
+        dequant_block_oscar2(b, y);
 }
 
 /* Head-row j of KV head h, dequantized into y[0..head_dim). */
@@ -272,8 +355,9 @@ static void dequant_row(const uint8_t *cache, int fmt, int head_dim, int64_t cap
                         int64_t j, double *y)
 {
     const uint8_t *r = cache + ((size_t)h * (size_t)capacity + (size_t)j) * row_bytes(fmt, head_dim);
-    for (int b = 0; b < head_dim / QK; ++b)
-        dequant_block(fmt, r + b * block_bytes(fmt), y + b * QK);
+    const int e = block_elems(fmt);
+    for (int b = 0; b < head_dim / e; ++b)
+        dequant_block(fmt, r + b * block_bytes(fmt), y + b * e);
 }
 
 /* Quantize-on-append: rows [pos, pos+n_tok) of every KV head.  k_new and
@@ -291,10 +375,11 @@ void orc_append(uint8_t *k_cache, uint8_t *v_cache, int n_kv_heads, int head_dim
             const size_t row = (size_t)h * capacity + (size_t)(pos + t);
             uint8_t *kd = k_cache + row * row_bytes(k_fmt, head_dim);
             uint8_t *vd = v_cache + row * row_bytes(v_fmt, head_dim);
-            for (int b = 0; b < head_dim / QK; ++b) {
-                quant_block(k_fmt, ks + b * QK, kd + b * block_bytes(k_fmt));
-                quant_block(v_fmt, vs + b * QK, vd + b * block_bytes(v_fmt));
-            }
+            const int ek = block_elems(k_fmt), ev = block_elems(v_fmt);
+            for (int b = 0; b < head_dim / ek; ++b)
+                quant_block(k_fmt, ks + b * ek, kd + b * block_bytes(k_fmt));
+            for (int b = 0; b < head_dim / ev; ++b)
+                quant_block(v_fmt, vs + b * ev, vd + b * block_bytes(v_fmt));
         }
 }
 

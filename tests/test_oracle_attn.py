@@ -260,10 +260,19 @@ def test_workload_generator_is_seeded_and_blockwise():
 # written and read in) is pinned against the separately pinned block
 # quantizers and dequantizers.
 
+O2 = oracle.FMT_OSCAR2
 FORMATS = [(oracle.FMT_Q8_0, oracle.FMT_Q8_0), (oracle.FMT_Q4_0, oracle.FMT_Q4_0),
-           (oracle.FMT_Q4_0, oracle.FMT_Q8_0)]
-_QUANT = {oracle.FMT_Q8_0: oracle.quantize_q8_0, oracle.FMT_Q4_0: oracle.quantize_q4_0}
-_DEQ = {oracle.FMT_Q8_0: oracle.dequant_q8_0, oracle.FMT_Q4_0: oracle.dequant_q4_0}
+           (oracle.FMT_Q4_0, oracle.FMT_Q8_0), (O2, O2), (oracle.FMT_Q8_0, O2),
+           (O2, oracle.FMT_Q4_0)]
+_QUANT = {oracle.FMT_Q8_0: oracle.quantize_q8_0, oracle.FMT_Q4_0: oracle.quantize_q4_0,
+          O2: oracle.quantize_oscar2}
+_DEQ = {oracle.FMT_Q8_0: oracle.dequant_q8_0, oracle.FMT_Q4_0: oracle.dequant_q4_0,
+        O2: oracle.dequant_oscar2}
+
+
+def _dim(k_fmt, v_fmt):
+    """head_dim of the format tests: 64, or 128 where an OSCAR2 tensor needs whole blocks."""
+    return 128 if O2 in (k_fmt, v_fmt) else 64
 
 
 def _fmt_cache(H, D, cap, k_fmt, v_fmt, seed):
@@ -278,7 +287,7 @@ def _fmt_cache(H, D, cap, k_fmt, v_fmt, seed):
 
 @pytest.mark.parametrize("k_fmt,v_fmt", FORMATS)
 def test_format_append_writes_each_tensors_blocks(k_fmt, v_fmt):
-    H, D, cap = 2, 64, 5
+    H, D, cap = 2, _dim(k_fmt, v_fmt), 5
     k, v, kc, vc = _fmt_cache(H, D, cap, k_fmt, v_fmt, 11)
     for h in range(H):
         assert np.array_equal(kc[h].reshape(-1), _QUANT[k_fmt](k[:, h].reshape(-1)))
@@ -287,7 +296,7 @@ def test_format_append_writes_each_tensors_blocks(k_fmt, v_fmt):
 
 @pytest.mark.parametrize("k_fmt,v_fmt", FORMATS)
 def test_format_single_key_and_brute_force(k_fmt, v_fmt):
-    H, D, Hq, T = 2, 64, 4, 2
+    H, D, Hq, T = 2, _dim(k_fmt, v_fmt), 4, 2
     n_kv = 9
     k, v, kc, vc = _fmt_cache(H, D, n_kv, k_fmt, v_fmt, 12)
     K = _DEQ[k_fmt](kc).reshape(H, n_kv, D)

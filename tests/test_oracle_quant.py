@@ -1,4 +1,4 @@
-"""Pins of the CPU oracle's fp16 conversion and Q8_0 / Q4_0 quantizers.
+"""Pins of the CPU oracle's fp16 conversion and Q8_0 / Q4_0 / OSCAR2 quantizers.
 
 Every expected value here comes from the pages (byte sizes), from a hand
 derivation of the quantizer definitions (golden blocks), from a library
@@ -58,6 +58,8 @@ def test_block_sizes_match_pages():
     x = np.zeros(128, np.float32)
     assert oracle.quantize_q8_0(x).size == s["q8_0_bytes_per_128"]
     assert np.zeros(128, np.float16).nbytes == s["f16_bytes_per_128"]
+    assert oracle.quantize_oscar2(x).size == s["oscar2_bytes_per_128"]
+    assert oracle.quantize_oscar2(x).size * 8 * 100 // 128 == s["oscar2_bits_per_elem_x100"]
     # 16 attention layers x 4 KV heads x 256: K as Q8_0 plus V as Q4_0
     row = np.zeros(4 * 256, np.float32)
     per_layer = oracle.quantize_q8_0(row).size + oracle.quantize_q4_0(row).size
@@ -109,8 +111,9 @@ def test_f16_to_f64_all_patterns_match_library():
 @pytest.mark.parametrize("case", _golden_blocks(), ids=lambda c: c[0])
 def test_golden_blocks(case):
     fmt, x, expected = case
-    assert x.size == 32
-    got = (oracle.quantize_q8_0 if fmt == "q8_0" else oracle.quantize_q4_0)(x)
+    assert x.size == (128 if fmt == "oscar2" else 32)
+    got = {"q8_0": oracle.quantize_q8_0, "q4_0": oracle.quantize_q4_0,
+           "oscar2": oracle.quantize_oscar2}[fmt](x)
     assert bytes(got) == expected
 
 
@@ -123,6 +126,14 @@ def test_golden_dequant():
     b = np.frombuffer(bytes.fromhex("00bc50bf" + "88" * 14), np.uint8)
     y = oracle.dequant_q4_0(b)
     assert y[0] == 8 and y[16] == 3 and y[1] == -7 and y[17] == -3 and y[2] == 0
+    # OSCAR2: d = 0.5 (0x3800), m = -1.25 (0xBD00); byte 0 = 0b11_10_01_00 holds codes
+    # 0, 1, 2, 3 of elements 0, 32, 64, 96; byte 5 = 0b00_00_00_11: element 5 -> u = 3
+    b = np.frombuffer(bytes.fromhex("0038 00bd e4 00 00 00 00 03".replace(" ", "") + "00" * 26),
+                      np.uint8)
+    y = oracle.dequant_oscar2(b)
+    assert y.size == 128
+    assert [y[0], y[32], y[64], y[96]] == [-1.25, -0.75, -0.25, 0.25]
+    assert y[5] == 0.25 and y[37] == -1.25 and y[1] == -1.25
 
 
 # ---------------------------------------------------------------- properties
@@ -172,11 +183,68 @@ def test_q4_0_round_trip_bound_and_clamp():
     assert np.allclose(xh[np.arange(x.shape[0]), first], -8 * d16[:, 0], rtol=0, atol=0)
 
 
-@pytest.mark.parametrize("fmt", ["q8_0", "q4_0"])
+def _oscar2_blocks(seed, n_blocks):
+    """128-element blocks: N(0,1) with 4 outlier elements x 8, block scales e^U(-8, 6)
+    (the minimum is stored as fp16, so every value stays well inside its range)."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((n_blocks, 128)).astype(np.float32)
+    x[:, rng.choice(128, 4, replace=False)] *= 8
+    scale = np.exp(rng.uniform(-8, 6, size=(n_blocks, 1))).astype(np.float32)
+    return (x * scale).astype(np.float32)
+
+
+def _dm(blocks):
+    b = blocks.reshape(-1, 36)
+    dm = b[:, :4].copy().view(np.float16).astype(np.float64)
+    return dm[:, 0:1], dm[:, 1:2]
+
+
+def test_oscar2_round_trip_bound():
+    """|x - x^| <= d/2 for the fp32 d and minimum the codes were chosen with, plus the
+    fp16 rounding of d (up to 3 steps) and of the minimum, plus fp32 rounding slack."""
+    x = _oscar2_blocks(4, 20000)
+    b = oracle.quantize_oscar2(x)
+    xh = oracle.dequant_oscar2(b).reshape(x.shape)
+    d16, m16 = _dm(b)
+    mn = x.min(axis=1, keepdims=True)
+    mx = x.max(axis=1, keepdims=True)
+    d32 = (((mx - mn).astype(np.float32)) / np.float32(3)).astype(np.float64)
+    slack = 3 * np.abs(d32 - d16) + np.abs(mn - m16) + 1e-6 * (np.abs(mx) + np.abs(mn))
+    assert (np.abs(x - xh) <= d32 / 2 + slack).all()
+    # the stored scale and zero-point are the fp16 roundings of d and of the minimum
+    assert (np.abs(d16 - d32) <= 2.0 ** -11 * d32 + 2.0 ** -25).all()
+    assert (np.abs(m16 - mn) <= 2.0 ** -11 * np.abs(mn) + 2.0 ** -25).all()
+    # the minimum decodes from code 0 and the maximum from code 3
+    codes = np.unpackbits(b.reshape(-1, 36)[:, 4:, None], axis=2, bitorder="little")
+    assert codes.shape == (x.shape[0], 32, 8)
+    u = (codes[:, :, 0::2] + 2 * codes[:, :, 1::2]).transpose(0, 2, 1).reshape(x.shape)
+    r = np.arange(x.shape[0])
+    assert (u[r, np.argmin(x, axis=1)] == 0).all() and (u[r, np.argmax(x, axis=1)] == 3).all()
+
+
+def test_oscar2_grid_values_round_trip_exactly():
+    """Blocks whose values lie on an fp16 grid m + d u with codes 0 and 3 present come
+    back exactly, and their codes are the grid indices."""
+    rng = np.random.default_rng(5)
+    n = 3000
+    d = np.float16(2.0) ** rng.integers(-12, 6, size=(n, 1)).astype(np.float16)
+    d = (d * rng.integers(1024, 2048, size=(n, 1)) / 1024).astype(np.float16)
+    m = (rng.integers(-64, 64, size=(n, 1)) * d.astype(np.float64)).astype(np.float16)
+    m = m.astype(np.float64)  # an fp16 zero-point within 64 steps of 0
+    u = rng.integers(0, 4, size=(n, 128))
+    u[:, 0], u[:, 127] = 0, 3
+    x = (m + d.astype(np.float64) * u).astype(np.float32)
+    assert np.array_equal(x.astype(np.float64), m + d.astype(np.float64) * u)  # exact inputs
+    b = oracle.quantize_oscar2(x)
+    assert np.array_equal(oracle.dequant_oscar2(b).reshape(x.shape), x.astype(np.float64))
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "oscar2"])
 def test_quantize_dequant_idempotent(fmt):
-    x = _random_blocks(3, 5000)
-    q, dq, nb = ((oracle.quantize_q8_0, oracle.dequant_q8_0, 34) if fmt == "q8_0"
-                 else (oracle.quantize_q4_0, oracle.dequant_q4_0, 18))
+    x = _oscar2_blocks(3, 2000) if fmt == "oscar2" else _random_blocks(3, 5000)
+    q, dq, nb = {"q8_0": (oracle.quantize_q8_0, oracle.dequant_q8_0, 34),
+                 "q4_0": (oracle.quantize_q4_0, oracle.dequant_q4_0, 18),
+                 "oscar2": (oracle.quantize_oscar2, oracle.dequant_oscar2, 36)}[fmt]
     b = q(x)
     d16 = np.abs(_d(b, nb))
     normal = d16 >= 2.0 ** -14  # fp16 normal scale: dequantized values re-quantize exactly
@@ -191,3 +259,4 @@ def test_zero_scale_block_dequantizes_to_zero():
     x = np.zeros(64, np.float32)
     assert (oracle.dequant_q8_0(oracle.quantize_q8_0(x)) == 0).all()
     assert (oracle.dequant_q4_0(oracle.quantize_q4_0(x)) == 0).all()
+    assert (oracle.dequant_oscar2(oracle.quantize_oscar2(np.zeros(256, np.float32))) == 0).all()
