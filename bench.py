@@ -49,9 +49,11 @@ from quantized_kv_long_b200 import workload as wl  # noqa: E402
 METRIC = "q8_0/q4_0 decode attn: KV GB/s (% of HBM peak), query-tok/s at 262k ctx"
 FALLBACK_HBM_GBS = 6650.0
 KV_BYTES_PER_TOKEN_LAYER = lambda w: w.n_kv_heads * (w.head_dim // 32) * (34 + 18)  # noqa: E731
-# --kv-formats: (K block type, V block type) of the C ABI and the bytes of one block of each
+# --kv-formats: (K block type, V block type) of the C ABI and the bytes per 32 elements of
+# each (OSCAR2: 36 B per 128 elements = 9 B per 32)
 KV_FORMATS = {"q8_0/q4_0": (1, 2, 34, 18), "q8_0/q8_0": (1, 1, 34, 34),
-              "q4_0/q4_0": (2, 2, 18, 18), "q4_0/q8_0": (2, 1, 18, 34)}
+              "q4_0/q4_0": (2, 2, 18, 18), "q4_0/q8_0": (2, 1, 18, 34),
+              "oscar2/oscar2": (3, 3, 9, 9), "q8_0/oscar2": (1, 3, 34, 9)}
 
 
 # --------------------------------------------------------------------------- helpers

@@ -43,6 +43,16 @@
  *        j in the low nibble and element j+16 in the high nibble; x^ = d*(u-8).
  *        m = the signed first element of largest |x|, d = m/-8,
  *        id = d ? 1/d : 0, u = min(15, trunc(x*id + 8.5)).
+ *  OSCAR2, 36 B per 128 elements (the INT2 format of the OSCAR2 page's
+ *        Compression Ratios table, 2.25 bits per element, with an fp16
+ *        zero-point): fp16 d, fp16 m, then 32 bytes; byte j holds the 2-bit
+ *        codes u of elements j, j+32, j+64, j+96 in bits 0-1, 2-3, 4-5, 6-7;
+ *        x^ = d*u + m.  mn = min x, mx = max x, d = (mx - mn)/3,
+ *        id = d ? 1/d : 0, u = min(3, trunc((x - mn)*id + 0.5)); m = fp16(mn).
+ *        A tensor in this format needs head_dim a multiple of 128, and its
+ *        values must lie inside the fp16 range (m is stored as fp16).  The
+ *        page's Hadamard rotation is baked into a model's weights before any
+ *        row reaches the cache; no call rotates.
  *  Only fp16(d) is stored; the quantizer divides by the fp32 d.
  *
  * Cache layout of one layer (head-major, fixed):
@@ -51,15 +61,17 @@
  *  V: [n_kv_heads][capacity][head_dim/32] Q4_0 blocks
  *     -> one head-row is head_dim/32*18 bytes (144 B at 256)
  *  That is the pages' configuration (kvq_layer k_type = v_type = 0).  Either
- *  tensor may instead use the other format (KVQ_TYPE_Q8_0 / KVQ_TYPE_Q4_0,
- *  the q8_0 and q4_0 choices of the KV-cache guide's levers section); its
- *  head-rows are then head_dim/32 blocks of that format.
+ *  tensor may instead use another format (KVQ_TYPE_Q8_0 / KVQ_TYPE_Q4_0, the
+ *  q8_0 and q4_0 choices of the KV-cache guide's levers section, or
+ *  KVQ_TYPE_OSCAR2); its head-rows are then head_dim / (elements per block)
+ *  blocks of that format (36*head_dim/128 bytes for OSCAR2).
  *  Head-rows of consecutive tokens of a head are contiguous, so a run of
  *  tokens is one contiguous byte range.  Both base pointers must be 16-byte
  *  aligned and capacity a multiple of 8: then every head starts on a 16-byte
- *  boundary (8 head-rows are 272*(head_dim/32) or 144*(head_dim/32) bytes),
+ *  boundary (8 head-rows are 272*(head_dim/32), 144*(head_dim/32) or
+ *  288*(head_dim/128) bytes),
  *  and so does every run of tokens that starts at a multiple of 8.
- *  head_dim is a multiple of 32, at most 512.
+ *  head_dim is a multiple of 32 (of 128 where a tensor is OSCAR2), at most 512.
  *
  * Attention (the plainest reading): query head g reads KV head
  * g / (n_q_heads / n_kv_heads); s_j = scale * sum_i q_i k^_ij;
@@ -102,7 +114,8 @@ typedef void *kvq_stream;
 typedef enum kvq_type {
     KVQ_TYPE_DEFAULT = 0,
     KVQ_TYPE_Q8_0 = 1,   /* 34 B per 32 elements */
-    KVQ_TYPE_Q4_0 = 2    /* 18 B per 32 elements */
+    KVQ_TYPE_Q4_0 = 2,   /* 18 B per 32 elements */
+    KVQ_TYPE_OSCAR2 = 3  /* 36 B per 128 elements (INT2, fp16 zero-point) */
 } kvq_type;
 
 typedef struct kvq_layer {
@@ -111,7 +124,8 @@ typedef struct kvq_layer {
     void *v;             /* V blocks, layout above                           */
     int64_t capacity;    /* tokens per head the two arrays hold              */
     int32_t n_kv_heads;  /* KV heads (4 in the pages' hybrid model)          */
-    int32_t head_dim;    /* elements per head-row, a multiple of 32, <= 512  */
+    int32_t head_dim;    /* elements per head-row, a multiple of 32 (128 for
+                            an OSCAR2 tensor), <= 512                        */
     int32_t k_type;      /* kvq_type of K (0: Q8_0)                          */
     int32_t v_type;      /* kvq_type of V (0: Q4_0)                          */
 } kvq_layer;
@@ -142,6 +156,17 @@ kvq_status kvq_quantize_q8_0(const float *x, void *blocks, int64_t n, kvq_stream
  * Arguments and errors as kvq_quantize_q8_0. */
 kvq_status kvq_quantize_q4_0(const float *x, void *blocks, int64_t n, kvq_stream stream);
 
+/* Quantize n fp32 values to OSCAR2 blocks (36 B per 128 elements).
+ * Source: Compression Ratios table of the OSCAR2 page (oscar2: 36 B per 128
+ * elements, 2.25 bits, INT2 with fp16 zero-point metadata); the bit layout
+ * and the rule are this library's reading (block formats above).
+ *  x      device, fp32[n], 4-byte aligned, values inside the fp16 range
+ *  blocks device, n/128 blocks of 36 bytes, written in order, 4-byte aligned
+ *  n      multiple of 128, >= 0 (0 launches nothing)
+ * Errors: INVALID_ARG (null pointer with n > 0, n % 128 != 0, n < 0),
+ *         ALIGNMENT (x or blocks not 4-byte aligned), CUDA. */
+kvq_status kvq_quantize_oscar2(const float *x, void *blocks, int64_t n, kvq_stream stream);
+
 /* Quantize-on-append of new K/V rows into rows [pos, pos+n_tok) of every KV
  * head of n_layers layers (K -> Q8_0, V -> Q4_0, or the layers' k_type /
  * v_type).
@@ -153,8 +178,9 @@ kvq_status kvq_quantize_q4_0(const float *x, void *blocks, int64_t n, kvq_stream
  *  pos     first row written; pos + n_tok <= capacity of every layer
  * Errors: INVALID_ARG (nulls, n_layers outside [1, KVQ_MAX_LAYERS], n_tok < 1,
  *         pos < 0, pos + n_tok > capacity, layers that differ in heads/dim,
- *         capacity % 8 != 0), ALIGNMENT, UNSUPPORTED (head_dim not a multiple
- *         of 32 or > 512), CUDA. */
+ *         capacity % 8 != 0, an unknown block type), ALIGNMENT, UNSUPPORTED
+ *         (head_dim not a multiple of 32, or of 128 for an OSCAR2 tensor, or
+ *         > 512), CUDA.  Every call that takes layers checks them the same way. */
 kvq_status kvq_append(const kvq_layer *layers, int n_layers, const float *k_new,
                       const float *v_new, int64_t pos, int n_tok, kvq_stream stream);
 

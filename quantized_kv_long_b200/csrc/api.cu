@@ -86,7 +86,7 @@ static kvq_status check_layers(const kvq_layer *layers, int n_layers, const char
     for (int l = 0; l < n_layers; ++l) {
         const kvq_layer &L = layers[l];
         for (const int t : {L.k_type, L.v_type})
-            if (t != KVQ_TYPE_DEFAULT && t != KVQ_TYPE_Q8_0 && t != KVQ_TYPE_Q4_0)
+            if (!known_type(t))
                 return set_error(KVQ_ERR_INVALID_ARG, "%s: layer %d has block type %d", fn, l, t);
         if (k_type_of(L) != k_type_of(layers[0]) || v_type_of(L) != v_type_of(layers[0]))
             return set_error(KVQ_ERR_INVALID_ARG, "%s: layer %d differs in block formats", fn, l);
@@ -100,6 +100,10 @@ static kvq_status check_layers(const kvq_layer *layers, int n_layers, const char
         if (!aligned(L.k, 16) || !aligned(L.v, 16))
             return set_error(KVQ_ERR_ALIGNMENT, "%s: layer %d cache not 16-byte aligned", fn, l);
     }
+    for (const int t : {k_type_of(layers[0]), v_type_of(layers[0])})
+        if (D % block_elems(t) != 0)
+            return set_error(KVQ_ERR_UNSUPPORTED, "%s: head_dim=%d is not a multiple of the "
+                             "%d-element OSCAR2 block", fn, D, block_elems(t));
     return KVQ_OK;
 }
 
@@ -258,6 +262,20 @@ kvq_status kvq_quantize_q4_0(const float *x, void *blocks, int64_t n, kvq_stream
     KVQ_TRY(need(x, 4, "x", fn));
     KVQ_TRY(need(static_cast<const uint8_t *>(blocks), 2, "blocks", fn));
     launch_quantize_q4_0(x, static_cast<uint8_t *>(blocks), n, as_stream(stream));
+    return check_launch(fn);
+}
+
+kvq_status kvq_quantize_oscar2(const float *x, void *blocks, int64_t n, kvq_stream stream)
+{
+    const char *fn = "kvq_quantize_oscar2";
+    if (n < 0 || n % QK_OSCAR2 != 0)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: n=%lld not a non-negative multiple of 128",
+                         fn, (long long)n);
+    if (n == 0)
+        return KVQ_OK;
+    KVQ_TRY(need(x, 4, "x", fn));
+    KVQ_TRY(need(static_cast<const uint8_t *>(blocks), 4, "blocks", fn));
+    launch_quantize_oscar2(x, static_cast<uint8_t *>(blocks), n, as_stream(stream));
     return check_launch(fn);
 }
 

@@ -6,29 +6,43 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "kvq.h"
 
 namespace kvq {
 
-constexpr int QK = 32;           // elements per quantization block
+constexpr int QK = 32;           // elements per Q8_0 / Q4_0 block
 constexpr int Q8_0_BYTES = 34;   // fp16 d + 32 x int8
 constexpr int Q4_0_BYTES = 18;   // fp16 d + 16 bytes of nibbles
+constexpr int QK_OSCAR2 = 128;   // elements per OSCAR2 block
+constexpr int OSCAR2_BYTES = 36; // fp16 d + fp16 m + 32 bytes of 2-bit codes
 
 __host__ __device__ inline int64_t k_row_bytes(int head_dim) { return (int64_t)(head_dim / QK) * Q8_0_BYTES; }
 __host__ __device__ inline int64_t v_row_bytes(int head_dim) { return (int64_t)(head_dim / QK) * Q4_0_BYTES; }
 
 // Block formats (kvq_type resolved: KVQ_TYPE_DEFAULT becomes Q8_0 for K, Q4_0 for V).
-__host__ __device__ inline int block_bytes(int type) { return type == KVQ_TYPE_Q8_0 ? Q8_0_BYTES : Q4_0_BYTES; }
-__host__ __device__ inline int64_t row_bytes(int type, int head_dim) { return (int64_t)(head_dim / QK) * block_bytes(type); }
+__host__ __device__ constexpr int block_elems(int type) { return type == KVQ_TYPE_OSCAR2 ? QK_OSCAR2 : QK; }
+__host__ __device__ constexpr int block_bytes(int type)
+{
+    return type == KVQ_TYPE_Q8_0 ? Q8_0_BYTES : type == KVQ_TYPE_Q4_0 ? Q4_0_BYTES : OSCAR2_BYTES;
+}
+__host__ __device__ inline int64_t row_bytes(int type, int head_dim)
+{
+    return (int64_t)(head_dim / block_elems(type)) * block_bytes(type);
+}
 
-// Integer value of element i (0..31) of a block: int8 q (Q8_0) or nibble - 8
-// (Q4_0: byte i holds element i in the low nibble and element i + 16 in the high).
+// Every block decodes as x^ = d * code + m.  Integer code of element i of a block:
+// int8 q (Q8_0); nibble - 8 (Q4_0: byte i holds element i in the low nibble and
+// element i + 16 in the high); the 2-bit u (OSCAR2: byte 4 + j holds elements j,
+// j + 32, j + 64, j + 96 in bits 0-1, 2-3, 4-5, 6-7).
 template <int TYPE>
 __device__ __forceinline__ int block_int(const uint8_t *blk, int i)
 {
     if (TYPE == KVQ_TYPE_Q8_0)
         return (int)(int8_t)blk[2 + i];
+    if (TYPE == KVQ_TYPE_OSCAR2)
+        return (blk[4 + (i & 31)] >> (2 * (i >> 5))) & 3;
     const uint8_t byte = blk[2 + (i & 15)];
     return (i < 16 ? (byte & 15) : (byte >> 4)) - 8;
 }
@@ -37,6 +51,48 @@ __device__ __forceinline__ int block_int(const uint8_t *blk, int i)
 __device__ __forceinline__ float block_d(const uint8_t *blk)
 {
     return __half2float(__ushort_as_half((unsigned short)(blk[0] | (blk[1] << 8))));
+}
+
+// The block's offset m as fp32: the fp16 zero-point in bytes 2-3 of an OSCAR2
+// block, 0 for the symmetric formats.
+template <int TYPE>
+__device__ __forceinline__ float block_m(const uint8_t *blk)
+{
+    if (TYPE != KVQ_TYPE_OSCAR2)
+        return 0.0f;
+    return __half2float(__ushort_as_half((unsigned short)(blk[2] | (blk[3] << 8))));
+}
+
+// Calls f(K, V) with K, V = std::integral_constant<int, format> for the resolved
+// formats kt, vt, so that a launcher can instantiate a kernel per format pair;
+// returns f's result, or false for an unknown format.
+template <typename F>
+bool launch_for_types(int kt, int vt, F &&f)
+{
+    using Q8 = std::integral_constant<int, KVQ_TYPE_Q8_0>;
+    using Q4 = std::integral_constant<int, KVQ_TYPE_Q4_0>;
+    using O2 = std::integral_constant<int, KVQ_TYPE_OSCAR2>;
+    auto with_v = [&](auto k) -> bool {
+        switch (vt) {
+        case KVQ_TYPE_Q8_0: return f(k, Q8{});
+        case KVQ_TYPE_Q4_0: return f(k, Q4{});
+        case KVQ_TYPE_OSCAR2: return f(k, O2{});
+        default: return false;
+        }
+    };
+    switch (kt) {
+    case KVQ_TYPE_Q8_0: return with_v(Q8{});
+    case KVQ_TYPE_Q4_0: return with_v(Q4{});
+    case KVQ_TYPE_OSCAR2: return with_v(O2{});
+    default: return false;
+    }
+}
+
+// Whether a block type is one of the formats (resolved or KVQ_TYPE_DEFAULT).
+inline bool known_type(int t)
+{
+    return t == KVQ_TYPE_DEFAULT || t == KVQ_TYPE_Q8_0 || t == KVQ_TYPE_Q4_0 ||
+           t == KVQ_TYPE_OSCAR2;
 }
 inline int k_type_of(const kvq_layer &l) { return l.k_type ? l.k_type : KVQ_TYPE_Q8_0; }
 inline int v_type_of(const kvq_layer &l) { return l.v_type ? l.v_type : KVQ_TYPE_Q4_0; }
@@ -107,6 +163,7 @@ inline cudaStream_t as_stream(kvq_stream s) { return reinterpret_cast<cudaStream
 // ---- launchers (host, internal) -------------------------------------------
 void launch_quantize_q8_0(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s);
 void launch_quantize_q4_0(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s);
+void launch_quantize_oscar2(const float *x, uint8_t *blocks, int64_t n, cudaStream_t s);
 void launch_append(const MutLayerTable &t, int n_layers, int n_kv_heads, int head_dim,
                    int k_type, int v_type, const float *k_new, const float *v_new, int64_t pos,
                    int n_tok, cudaStream_t s);
@@ -118,7 +175,7 @@ void launch_merge_lse_parts(const float *out_parts, const float *lse_parts, int 
 struct DecodeArgs {
     LayerTable layers;
     int n_layers, n_kv_heads, head_dim, n_q_heads, T;
-    int k_type, v_type;  // resolved block formats (KVQ_TYPE_Q8_0 / KVQ_TYPE_Q4_0)
+    int k_type, v_type;  // resolved block formats (KVQ_TYPE_Q8_0 / _Q4_0 / _OSCAR2)
     int64_t n_kv;
     // causal visibility: the row of token t sees the keys (rows of the layers) j <=
     // vis_last + t; n_kv - T for a whole context, less for a shard of one
@@ -162,7 +219,7 @@ struct PrefillArgs {
     unsigned int *status;
     int test_timeout;  // test hook: one bounded wait of each tensor-core launch runs out
     int pair0;         // first (layer, KV head) pair, layer * n_kv_heads + head, of a launch
-    int k_type, v_type;  // block formats (KVQ_TYPE_Q8_0 / KVQ_TYPE_Q4_0)
+    int k_type, v_type;  // block formats (KVQ_TYPE_Q8_0 / _Q4_0 / _OSCAR2)
 };
 size_t prefill_workspace_bytes(int n_layers, int n_q_heads, int n_kv_heads, int T, int head_dim);
 // Optional workspace of the tensor-core path: the f16 key tiles expanded once per

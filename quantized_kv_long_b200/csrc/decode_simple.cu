@@ -15,8 +15,9 @@
 // j <= vis_last + t (n_kv - T + t for a whole context) of chunk c = keys
 // [c*chunk, (c+1)*chunk).
 //
-// K and V may each be in either block format (template parameters KT, VT:
-// KVQ_TYPE_Q8_0 or KVQ_TYPE_Q4_0); the pages' configuration is Q8_0 K / Q4_0 V.
+// K and V may each be in any block format (template parameters KT, VT:
+// KVQ_TYPE_Q8_0, KVQ_TYPE_Q4_0 or KVQ_TYPE_OSCAR2, whose zero-point m enters
+// the score as m * sum(q) per block); the pages' configuration is Q8_0 K / Q4_0 V.
 #include "common.cuh"
 
 namespace kvq {
@@ -32,7 +33,8 @@ decode_simple_kernel(DecodeArgs a)
     const int G = a.n_q_heads / a.n_kv_heads;
     const int R = G * a.T;
     const int D = a.head_dim;
-    const int nb = D / QK;
+    constexpr int KE = block_elems(KT), VE = block_elems(VT);  // elements per block
+    const int nb = D / KE;
     float *q_s = sm;                       // [R][D]
     float *acc = q_s + R * D;              // [R][D]
     float *p_s = acc + R * D;              // [R][TILE]
@@ -73,10 +75,15 @@ decode_simple_kernel(DecodeArgs a)
                 float tot = 0.0f;
                 for (int b = 0; b < nb; ++b) {
                     const uint8_t *blk = kr + b * block_bytes(KT);
-                    float part = 0.0f;
-                    for (int i = 0; i < QK; ++i)
-                        part += qr[b * QK + i] * (float)block_int<KT>(blk, i);
+                    float part = 0.0f, qsum = 0.0f;
+                    for (int i = 0; i < KE; ++i) {
+                        part += qr[b * KE + i] * (float)block_int<KT>(blk, i);
+                        if (KT == KVQ_TYPE_OSCAR2)
+                            qsum += qr[b * KE + i];
+                    }
                     tot += block_d(blk) * part;
+                    if (KT == KVQ_TYPE_OSCAR2)  // q . (d u + m) = d (q . u) + m sum(q)
+                        tot += block_m<KT>(blk) * qsum;
                 }
                 s = a.scale * tot;
             }
@@ -111,14 +118,14 @@ decode_simple_kernel(DecodeArgs a)
         // 3. rescale and accumulate the weighted V rows
         for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
             const int r = p / D, i = p % D;
-            const int b = i / QK, ii = i % QK;
+            const int b = i / VE, ii = i % VE;
             float o = acc[p] * al_s[r];
             for (int jj = 0; jj < SIMPLE_TILE; ++jj) {
                 const float pw = p_s[r * SIMPLE_TILE + jj];
                 if (pw == 0.0f)
                     continue;
                 const uint8_t *blk = vb + (j0 + jj) * vrow + b * block_bytes(VT);
-                o += pw * (block_d(blk) * (float)block_int<VT>(blk, ii));
+                o += pw * (block_d(blk) * (float)block_int<VT>(blk, ii) + block_m<VT>(blk));
             }
             acc[p] = o;
         }
@@ -161,16 +168,9 @@ bool launch_decode_simple(const DecodeArgs &a, cudaStream_t s)
     const size_t smem = decode_simple_smem(R, a.head_dim);
     if (smem > 227 * 1024)
         return false;
-    constexpr int Q8 = KVQ_TYPE_Q8_0, Q4 = KVQ_TYPE_Q4_0;
-    if (a.k_type == Q8 && a.v_type == Q4)
-        return launch_simple_typed<Q8, Q4>(a, smem, s);
-    if (a.k_type == Q8 && a.v_type == Q8)
-        return launch_simple_typed<Q8, Q8>(a, smem, s);
-    if (a.k_type == Q4 && a.v_type == Q4)
-        return launch_simple_typed<Q4, Q4>(a, smem, s);
-    if (a.k_type == Q4 && a.v_type == Q8)
-        return launch_simple_typed<Q4, Q8>(a, smem, s);
-    return false;
+    return launch_for_types(a.k_type, a.v_type, [&](auto kt, auto vt) {
+        return launch_simple_typed<decltype(kt)::value, decltype(vt)::value>(a, smem, s);
+    });
 }
 
 }  // namespace kvq

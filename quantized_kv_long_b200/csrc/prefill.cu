@@ -795,7 +795,8 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
 {
     extern __shared__ float ex_sm[];
     const int G = a.n_q_heads / a.n_kv_heads;
-    const int D = a.head_dim, nb = D / QK;
+    constexpr int KE = block_elems(KT), VE = block_elems(VT);  // elements per block
+    const int D = a.head_dim, nb = D / KE;
     const int t0 = blockIdx.x * tb_tok;
     const int ntok = min(tb_tok, t_end - t0);
     const int R = ntok * G;
@@ -860,10 +861,15 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
                 float tot = 0.0f;
                 for (int bq = 0; bq < nb; ++bq) {
                     const uint8_t *blk = kr + bq * block_bytes(KT);
-                    float part = 0.0f;
-                    for (int i = 0; i < QK; ++i)
-                        part += qr[bq * QK + i] * (float)block_int<KT>(blk, i);
+                    float part = 0.0f, qsum = 0.0f;
+                    for (int i = 0; i < KE; ++i) {
+                        part += qr[bq * KE + i] * (float)block_int<KT>(blk, i);
+                        if (KT == KVQ_TYPE_OSCAR2)
+                            qsum += qr[bq * KE + i];
+                    }
                     tot += block_d(blk) * part;
+                    if (KT == KVQ_TYPE_OSCAR2)  // q . (d u + m) = d (q . u) + m sum(q)
+                        tot += block_m<KT>(blk) * qsum;
                 }
                 s = a.scale * tot;
             }
@@ -895,14 +901,14 @@ __global__ void __launch_bounds__(EX_THREADS) prefill_exact_kernel(const Prefill
         __syncthreads();
         for (int p = threadIdx.x; p < R * D; p += blockDim.x) {
             const int r = p / D, i = p % D;
-            const int bq = i / QK, ii = i % QK;
+            const int bq = i / VE, ii = i % VE;
             float o = acc[p] * al_s[r];
             for (int jj = 0; jj < EX_TILE; ++jj) {
                 const float pw = p_s[r * EX_TILE + jj];
                 if (pw == 0.0f)
                     continue;
                 const uint8_t *blk = vb + (j0 + jj) * vrow + bq * block_bytes(VT);
-                o += pw * (block_d(blk) * (float)block_int<VT>(blk, ii));
+                o += pw * (block_d(blk) * (float)block_int<VT>(blk, ii) + block_m<VT>(blk));
             }
             acc[p] = o;
         }
@@ -1010,15 +1016,11 @@ bool launch_prefill(const PrefillArgs &a_in, cudaStream_t s)
         const size_t smem = sizeof(float) * ((size_t)2 * tb * G * a.head_dim +
                                              (size_t)tb * G * EX_TILE + 3 * (size_t)tb * G);
         dim3 grid((unsigned)((t_split + tb - 1) / tb), a.n_kv_heads, a.n_layers);
-        constexpr int Q8 = KVQ_TYPE_Q8_0, Q4 = KVQ_TYPE_Q4_0;
-        if (a.k_type == Q8 && a.v_type == Q4)
-            launch_exact<Q8, Q4>(a, grid, smem, tb, (int)t_split, s);
-        else if (a.k_type == Q8 && a.v_type == Q8)
-            launch_exact<Q8, Q8>(a, grid, smem, tb, (int)t_split, s);
-        else if (a.k_type == Q4 && a.v_type == Q4)
-            launch_exact<Q4, Q4>(a, grid, smem, tb, (int)t_split, s);
-        else
-            launch_exact<Q4, Q8>(a, grid, smem, tb, (int)t_split, s);
+        launch_for_types(a.k_type, a.v_type, [&](auto kt, auto vt) {
+            launch_exact<decltype(kt)::value, decltype(vt)::value>(a, grid, smem, tb,
+                                                                   (int)t_split, s);
+            return true;
+        });
     }
     if (t_split == a.T)
         return true;

@@ -194,9 +194,11 @@ extern "C" int kvq_resident_layers(size_t budget_bytes, int n_layers, int64_t ca
     if (n_layers < 1 || capacity < 1 || n_kv_heads < 1 || head_dim < QK || head_dim % QK != 0)
         return -1;
     for (const int t : {k_type, v_type})
-        if (t != KVQ_TYPE_DEFAULT && t != KVQ_TYPE_Q8_0 && t != KVQ_TYPE_Q4_0)
+        if (!known_type(t))
             return -1;
     const int kt = k_type ? k_type : KVQ_TYPE_Q8_0, vt = v_type ? v_type : KVQ_TYPE_Q4_0;
+    if (head_dim % block_elems(kt) != 0 || head_dim % block_elems(vt) != 0)
+        return -1;
     const double layer = (double)n_kv_heads * (double)capacity *
                          (double)(row_bytes(kt, head_dim) + row_bytes(vt, head_dim));
     const double budget = (double)budget_bytes;

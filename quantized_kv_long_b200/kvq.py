@@ -42,14 +42,30 @@ KVQ_MAX_DECODE_T = 4
 KVQ_STATIC_SCRATCH_BYTES = 8 << 20
 
 QK, Q8_0_BYTES, Q4_0_BYTES = 32, 34, 18
-KVQ_TYPE_DEFAULT, KVQ_TYPE_Q8_0, KVQ_TYPE_Q4_0 = 0, 1, 2
+QK_OSCAR2, OSCAR2_BYTES = 128, 36
+KVQ_TYPE_DEFAULT, KVQ_TYPE_Q8_0, KVQ_TYPE_Q4_0, KVQ_TYPE_OSCAR2 = 0, 1, 2, 3
+
+
+def _resolve(kvq_type: int, tensor: str) -> int:
+    if kvq_type == KVQ_TYPE_DEFAULT:
+        return KVQ_TYPE_Q8_0 if tensor == "k" else KVQ_TYPE_Q4_0
+    return kvq_type
 
 
 def block_bytes(kvq_type: int, tensor: str) -> int:
-    """Bytes per 32-element block of a cache tensor ('k' or 'v') in ``kvq_type``."""
-    if kvq_type == KVQ_TYPE_DEFAULT:
-        kvq_type = KVQ_TYPE_Q8_0 if tensor == "k" else KVQ_TYPE_Q4_0
-    return Q8_0_BYTES if kvq_type == KVQ_TYPE_Q8_0 else Q4_0_BYTES
+    """Bytes per block of a cache tensor ('k' or 'v') in ``kvq_type``."""
+    return {KVQ_TYPE_Q8_0: Q8_0_BYTES, KVQ_TYPE_Q4_0: Q4_0_BYTES,
+            KVQ_TYPE_OSCAR2: OSCAR2_BYTES}[_resolve(kvq_type, tensor)]
+
+
+def block_elems(kvq_type: int, tensor: str) -> int:
+    """Elements per block of a cache tensor ('k' or 'v') in ``kvq_type``."""
+    return QK_OSCAR2 if _resolve(kvq_type, tensor) == KVQ_TYPE_OSCAR2 else QK
+
+
+def row_bytes(kvq_type: int, tensor: str, head_dim: int) -> int:
+    """Bytes of one head-row of a cache tensor ('k' or 'v') in ``kvq_type``."""
+    return head_dim // block_elems(kvq_type, tensor) * block_bytes(kvq_type, tensor)
 
 
 class kvq_layer(ctypes.Structure):
@@ -75,6 +91,7 @@ _LP = ctypes.POINTER(kvq_layer)
 _SIGS = {
     "kvq_quantize_q8_0": ([_P, _P, _I64, _P], _I32),
     "kvq_quantize_q4_0": ([_P, _P, _I64, _P], _I32),
+    "kvq_quantize_oscar2": ([_P, _P, _I64, _P], _I32),
     "kvq_append": ([_LP, _I32, _P, _P, _I64, _I32, _P], _I32),
     "kvq_decode_attn": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P], _I32),
     "kvq_merge_lse": ([_P, _P, _I64, _I32, _I32, _P, _P, _P], _I32),
@@ -158,6 +175,11 @@ def kvq_quantize_q8_0(x, blocks, n: int | None = None, stream=None) -> None:
 def kvq_quantize_q4_0(x, blocks, n: int | None = None, stream=None) -> None:
     n = x.numel() if n is None else n
     _check(_lib.kvq_quantize_q4_0(_ptr(x), _ptr(blocks), n, _stream(stream)))
+
+
+def kvq_quantize_oscar2(x, blocks, n: int | None = None, stream=None) -> None:
+    n = x.numel() if n is None else n
+    _check(_lib.kvq_quantize_oscar2(_ptr(x), _ptr(blocks), n, _stream(stream)))
 
 
 def kvq_append(layers, k_new, v_new, pos: int, n_tok: int, stream=None) -> None:
@@ -287,7 +309,8 @@ class QuantizedKVCache:
 
     K of layer ``l``: uint8 ``[n_kv_heads, capacity, head_dim // 32 * 34]``;
     V: ``[n_kv_heads, capacity, head_dim // 32 * 18]`` (the default Q8_0 K /
-    Q4_0 V; ``k_type`` / ``v_type`` select the other block format per tensor).
+    Q4_0 V; ``k_type`` / ``v_type`` select another block format per tensor:
+    Q8_0, Q4_0 or OSCAR2, ``head_dim // 128 * 36`` bytes per head-row).
     ``device="cpu"`` with ``pin=True`` gives pinned host memory for
     :func:`kvq_stream_decode`.
     """
@@ -300,8 +323,8 @@ class QuantizedKVCache:
         self.n_layers, self.n_kv_heads, self.head_dim, self.capacity = (
             n_layers, n_kv_heads, head_dim, capacity)
         self.k_type, self.v_type = k_type, v_type
-        kb = head_dim // QK * block_bytes(k_type, "k")
-        vb = head_dim // QK * block_bytes(v_type, "v")
+        kb = row_bytes(k_type, "k", head_dim)
+        vb = row_bytes(v_type, "v", head_dim)
         kw = dict(dtype=torch.uint8, device=device)
         if pin:
             kw["pin_memory"] = True

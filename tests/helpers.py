@@ -39,7 +39,8 @@ def oracle_fmt(kvq, kvq_type: int, tensor: str) -> int:
     """The oracle's block format for a kvq_type of a cache tensor ('k' or 'v')."""
     if kvq_type == kvq.KVQ_TYPE_DEFAULT:
         return oracle.FMT_Q8_0 if tensor == "k" else oracle.FMT_Q4_0
-    return {kvq.KVQ_TYPE_Q8_0: oracle.FMT_Q8_0, kvq.KVQ_TYPE_Q4_0: oracle.FMT_Q4_0}[kvq_type]
+    return {kvq.KVQ_TYPE_Q8_0: oracle.FMT_Q8_0, kvq.KVQ_TYPE_Q4_0: oracle.FMT_Q4_0,
+            kvq.KVQ_TYPE_OSCAR2: oracle.FMT_OSCAR2}[kvq_type]
 
 
 def fill_both(w: wl.Workload, layers, n_rows: int, capacity: int, device="cuda", k_type=0,

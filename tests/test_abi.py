@@ -64,6 +64,11 @@ def test_quantize_validation(kvq):
     _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_quantize_q4_0, A + 2, A, 64, 0)
     _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_quantize_q8_0, A, A + 1, 64, 0)
     kvq.kvq_quantize_q8_0(None, None, 0, 0)  # n == 0 launches nothing
+    # OSCAR2: whole 128-element blocks, 4-byte aligned blocks (two fp16 words)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_quantize_oscar2, A, A, 96, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_quantize_oscar2, None, A, 128, 0)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_quantize_oscar2, A, A + 2, 128, 0)
+    kvq.kvq_quantize_oscar2(None, None, 0, 0)
 
 
 def test_append_validation(kvq):
@@ -207,7 +212,7 @@ def test_resident_layers_plan(kvq):
 def test_block_format_validation(kvq):
     """Block formats: unknown types and layers that differ are refused (prefill
     included); the residency plan sizes layers by format."""
-    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, _layer(kvq, k_type=3), A, A, 0, 1, 0)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, _layer(kvq, k_type=4), A, A, 0, 1, 0)
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_append, _layer(kvq, v_type=-1), A, A, 0, 1, 0)
     # explicit Q8_0 K / Q4_0 V equals the default pair, so these two layers agree
     mixed_ok = [_layer(kvq), _layer(kvq, k_type=kvq.KVQ_TYPE_Q8_0, v_type=kvq.KVQ_TYPE_Q4_0)]
@@ -218,10 +223,22 @@ def test_block_format_validation(kvq):
     _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_prefill_attn,
             [_layer(kvq, v_type=1, capacity=4096), _layer(kvq, capacity=4096)],
             A, 24, 128, 1024, 1024, 1 / 16, A, A)
+    # an OSCAR2 tensor needs whole 128-element blocks in a head-row
+    O2 = kvq.KVQ_TYPE_OSCAR2
+    for call in (lambda L: kvq.kvq_append(L, A, A, 0, 1, 0),
+                 lambda L: kvq.kvq_decode_attn(L, A, 4, 1, 1024, 256, 1 / 16, A, A, 0),
+                 lambda L: kvq.kvq_prefill_attn(L, A, 4, 128, 512, 1024, 1 / 16, A, A)):
+        _raises(kvq, kvq.KVQ_ERR_UNSUPPORTED, call, _layer(kvq, head_dim=96, v_type=O2))
+        _raises(kvq, kvq.KVQ_ERR_UNSUPPORTED, call, _layer(kvq, head_dim=320, k_type=O2))
     q8 = 4 * 262144 * (272 + 272)
     assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 1, 1) == 3
     assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 0, 0) == 4
     assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, 7, 0) == -1
+    # OSCAR2 K and V head-rows of 72 B each: the bytes of 3 Q8_0/Q8_0 layers hold 11.3
+    # OSCAR2 layers, 9 of them beside the 2 streaming slots; 5 hold all 16
+    assert kvq.kvq_resident_layers(3 * q8, 16, 262144, 4, 256, O2, O2) == 9
+    assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 256, O2, O2) == 16
+    assert kvq.kvq_resident_layers(5 * q8, 16, 262144, 4, 96, O2, O2) == -1
 
 
 def test_prefill_workspace_validation(kvq):

@@ -1,8 +1,9 @@
 """Other block formats of the cache (Q8_0 or Q4_0 for each of K and V, the
-choices of the KV-cache guide's levers section) on the GPU, against the oracle.
+choices of the KV-cache guide's levers section, and the OSCAR2 page's INT2
+block) on the GPU, against the oracle.
 
 The default pair (Q8_0 K / Q4_0 V) is covered by the other GPU tests; here
-the three other pairs go through append (bit-exact cache bytes), the general
+five other pairs go through append (bit-exact cache bytes), the general
 decode kernel and the merge (tolerances of helpers.py), the decode step
 (bit-identical to the separate calls), the streamed decode (bit-identical to
 the resident one) and prefill (the exact kernel, which serves every pair).
@@ -25,7 +26,9 @@ def kvq():
     return m
 
 
-PAIRS = [(1, 1), (2, 2), (2, 1)]  # (k_type, v_type): q8_0/q8_0, q4_0/q4_0, q4_0/q8_0
+# (k_type, v_type): q8_0/q8_0, q4_0/q4_0, q4_0/q8_0, oscar2/oscar2 (the OSCAR2 page's
+# cache), q8_0/oscar2
+PAIRS = [(1, 1), (2, 2), (2, 1), (3, 3), (1, 3)]
 
 
 @pytest.mark.parametrize("k_type,v_type", PAIRS)

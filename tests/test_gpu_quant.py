@@ -9,7 +9,7 @@ import oracle
 from quantized_kv_long_b200 import workload as wl
 
 from helpers import fill_both
-from test_oracle_quant import _golden_blocks, _random_blocks
+from test_oracle_quant import _golden_blocks, _oscar2_blocks, _random_blocks
 
 pytestmark = pytest.mark.gpu
 
@@ -21,10 +21,15 @@ def kvq():
 
 
 def _gpu_quant(kvq, x, q8):
+    """Blocks of x on the GPU: Q8_0 if q8 is True, Q4_0 if False, OSCAR2 if "oscar2"."""
     xt = torch.from_numpy(np.ascontiguousarray(x, np.float32)).cuda()
-    nb = x.size // 32
-    out = torch.empty(nb * (34 if q8 else 18), dtype=torch.uint8, device="cuda")
-    (kvq.kvq_quantize_q8_0 if q8 else kvq.kvq_quantize_q4_0)(xt, out)
+    if q8 == "oscar2":
+        out = torch.empty(x.size // 128 * 36, dtype=torch.uint8, device="cuda")
+        kvq.kvq_quantize_oscar2(xt, out)
+    else:
+        nb = x.size // 32
+        out = torch.empty(nb * (34 if q8 else 18), dtype=torch.uint8, device="cuda")
+        (kvq.kvq_quantize_q8_0 if q8 else kvq.kvq_quantize_q4_0)(xt, out)
     torch.cuda.synchronize()
     return out.cpu().numpy()
 
@@ -49,7 +54,7 @@ def test_golden_and_edge_blocks_bit_exact(kvq):
         np.array([0.5 * (i % 2 * 2 - 1) for i in range(32)], np.float32),
     ]
     for fmt, x, expected in cases:
-        got = _gpu_quant(kvq, x, fmt == "q8_0")
+        got = _gpu_quant(kvq, x, "oscar2" if fmt == "oscar2" else fmt == "q8_0")
         assert bytes(got) == expected, fmt
     for x in edge:
         assert np.array_equal(_gpu_quant(kvq, x, True), oracle.quantize_q8_0(x))
@@ -70,6 +75,33 @@ def test_ties_at_half_bit_exact(kvq):
                         rng.integers(-7, 8, size=(n, 31)).astype(np.float32) + 0.5], axis=1)
     y = (y * scale).astype(np.float32)
     assert np.array_equal(_gpu_quant(kvq, y, False), oracle.quantize_q4_0(y))
+
+
+def test_oscar2_blocks_bit_exact(kvq):
+    """OSCAR2 on the GPU against the oracle: random blocks, grid blocks with exact
+    ties at .5 after the scale, and edge blocks (signed zeros, constants, a minimum
+    or maximum that occurs twice, values near the fp16 limits)."""
+    x = _oscar2_blocks(11, 100000)
+    assert np.array_equal(_gpu_quant(kvq, x, "oscar2"), oracle.quantize_oscar2(x))
+    rng = np.random.default_rng(12)
+    n = 4096
+    u2 = rng.integers(0, 7, size=(n, 128)).astype(np.float32) / 2  # codes and half-codes
+    u2[:, 5], u2[:, 77] = 0.0, 3.0
+    scale = (2.0 ** rng.integers(-8, 8, size=(n, 1))).astype(np.float32)
+    y = (u2 * scale + rng.integers(-4, 4, size=(n, 1)).astype(np.float32) * scale)
+    y = y.astype(np.float32)
+    assert np.array_equal(_gpu_quant(kvq, y, "oscar2"), oracle.quantize_oscar2(y))
+    z = np.zeros(128, np.float32)
+    mixed = z.copy()
+    mixed[::3] = -0.0                                     # -0 and +0: the first one wins
+    edge = [z, -z, mixed, -mixed, np.full(128, -7.25, np.float32),
+            np.concatenate([[2.0], np.zeros(126), [2.0]]).astype(np.float32),
+            np.concatenate([[-1.0], np.ones(126), [-1.0]]).astype(np.float32),
+            np.linspace(-60000, 60000, 128, dtype=np.float32),
+            np.full(128, 1e-30, np.float32),
+            (np.arange(128, dtype=np.float32) - 64) * np.float32(2.0 ** -20)]
+    for e in edge:
+        assert np.array_equal(_gpu_quant(kvq, e, "oscar2"), oracle.quantize_oscar2(e))
 
 
 @pytest.mark.parametrize("D,H,n_rows,cap", [(256, 4, 1024, 1024), (128, 2, 77, 80),
