@@ -256,3 +256,18 @@ def test_prefill_workspace_validation(kvq):
             ws_bytes=need - 1)
     _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_prefill_attn, *args, workspace=A + 16,
             ws_bytes=need)
+
+
+def test_cache_row_sizes_per_format(kvq):
+    """Head-row bytes of each block format, as the cache helper allocates them (host
+    memory here): 34, 18 and 9 bytes per 32 elements; OSCAR2 needs whole 128-element
+    blocks."""
+    assert kvq.row_bytes(kvq.KVQ_TYPE_DEFAULT, "k", 256) == 272
+    assert kvq.row_bytes(kvq.KVQ_TYPE_DEFAULT, "v", 256) == 144
+    assert kvq.row_bytes(kvq.KVQ_TYPE_OSCAR2, "k", 256) == 72
+    assert kvq.row_bytes(kvq.KVQ_TYPE_OSCAR2, "v", 512) == 144
+    c = kvq.QuantizedKVCache(2, 4, 256, 16, device="cpu", k_type=kvq.KVQ_TYPE_Q8_0,
+                             v_type=kvq.KVQ_TYPE_OSCAR2)
+    assert tuple(c.k[0].shape) == (4, 16, 272) and tuple(c.v[1].shape) == (4, 16, 72)
+    assert c.nbytes == 2 * 4 * 16 * (272 + 72)
+    assert (c.layer(1).k_type, c.layer(1).v_type) == (1, 3)
