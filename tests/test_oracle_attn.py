@@ -319,3 +319,29 @@ def test_format_single_key_and_brute_force(k_fmt, v_fmt):
             ref = (w / w.sum()) @ V[h, :n]
             assert np.allclose(out[t, g, 0], ref, rtol=0, atol=1e-12)
             assert abs(lse[t, g, 0] - (s.max() + math.log(w.sum()))) < 1e-12
+
+
+@pytest.mark.parametrize("k_fmt,v_fmt", [(O2, O2), (oracle.FMT_Q8_0, O2)])
+def test_format_prefill_equals_decode_and_brute_force(k_fmt, v_fmt):
+    """Prefill over OSCAR2 caches: each token's row equals a decode over the keys it
+    sees, the page partials merge to the one-pass rows, and both equal softmax
+    attention over the dequantized rows."""
+    H, Hq, D, n_cached, T, page = 2, 4, 128, 37, 5, 16
+    k, v, kc, vc = _fmt_cache(H, D, n_cached + T, k_fmt, v_fmt, 53)
+    K = _DEQ[k_fmt](kc).reshape(H, n_cached + T, D)
+    V = _DEQ[v_fmt](vc).reshape(H, n_cached + T, D)
+    q = _q(T, Hq, D, 54)
+    out, lse, po, pl = oracle.prefill_attn(kc, vc, q, n_cached, page, SCALE, pages=True)
+    mo, ml = oracle.merge_lse(po, pl)
+    assert np.allclose(mo, out, rtol=0, atol=1e-12) and np.allclose(ml, lse, rtol=0, atol=1e-12)
+    for t in range(T):
+        d, dl = oracle.decode_attn(kc, vc, q[t:t + 1], n_kv=n_cached + t + 1, chunk=1 << 20,
+                                   scale=SCALE)
+        assert np.allclose(out[t], d[0, :, 0], rtol=0, atol=1e-12)
+        for g in range(Hq):
+            h = g // (Hq // H)
+            n = n_cached + t + 1
+            s = SCALE * (K[h, :n] @ q[t, g].astype(np.float64))
+            w = np.exp(s - s.max())
+            assert np.allclose(out[t, g], (w / w.sum()) @ V[h, :n], rtol=0, atol=1e-12)
+            assert abs(lse[t, g] - (s.max() + math.log(w.sum()))) < 1e-12
