@@ -18,9 +18,6 @@ constexpr int Q4_0_BYTES = 18;   // fp16 d + 16 bytes of nibbles
 constexpr int QK_OSCAR2 = 128;   // elements per OSCAR2 block
 constexpr int OSCAR2_BYTES = 36; // fp16 d + fp16 m + 32 bytes of 2-bit codes
 
-__host__ __device__ inline int64_t k_row_bytes(int head_dim) { return (int64_t)(head_dim / QK) * Q8_0_BYTES; }
-__host__ __device__ inline int64_t v_row_bytes(int head_dim) { return (int64_t)(head_dim / QK) * Q4_0_BYTES; }
-
 // Block formats (kvq_type resolved: KVQ_TYPE_DEFAULT becomes Q8_0 for K, Q4_0 for V).
 __host__ __device__ constexpr int block_elems(int type) { return type == KVQ_TYPE_OSCAR2 ? QK_OSCAR2 : QK; }
 __host__ __device__ constexpr int block_bytes(int type)
