@@ -292,6 +292,29 @@ kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k
                            float *lse_part, float *out, float *lse, void *workspace,
                            size_t ws_bytes, kvq_stream stream);
 
+/* kvq_decode_step with the step's inputs and results in host memory: copies
+ * q_host, k_host and v_host into the device buffers q, k_new and v_new, runs
+ * the step (append, decode, merge), and copies out and lse back into out_host
+ * and lse_host -- five cudaMemcpyAsync and three launches, in that order on
+ * `stream`.  The host results are valid once the stream reaches the end of the
+ * call (kvq_check or a stream synchronisation).  Host buffers should be
+ * pinned: pageable memory makes the copies synchronous.
+ *  k_host, v_host  host fp32 [n_layers][T][n_kv_heads][head_dim]
+ *  q_host          host fp16 bits [n_layers][T][n_q_heads][head_dim]
+ *  out_host        host fp32 [n_layers][T][n_q_heads][head_dim]
+ *  lse_host        host fp32 [n_layers][T][n_q_heads]
+ *  k_new, v_new, q device buffers of those sizes (the copies' targets)
+ *  the rest        as kvq_decode_step (the workspace is not needed)
+ * Errors: INVALID_ARG (a NULL host buffer), those of kvq_decode_step (all
+ *         checked before the first copy), COPY (a copy could not be enqueued;
+ *         the copies and launches before it stay enqueued). */
+kvq_status kvq_decode_step_host(const kvq_layer *layers, int n_layers, const float *k_host,
+                                const float *v_host, const uint16_t *q_host, float *out_host,
+                                float *lse_host, float *k_new, float *v_new, uint16_t *q,
+                                int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                                float *out_part, float *lse_part, float *out, float *lse,
+                                kvq_stream stream);
+
 /* ---------------------------------------------------------------------- */
 /* Chunked prefill                                                         */
 /* ---------------------------------------------------------------------- */

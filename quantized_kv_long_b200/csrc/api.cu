@@ -390,6 +390,51 @@ kvq_status kvq_decode_step(const kvq_layer *layers, int n_layers, const float *k
     return check_launch(fn);
 }
 
+kvq_status kvq_decode_step_host(const kvq_layer *layers, int n_layers, const float *k_host,
+                                const float *v_host, const uint16_t *q_host, float *out_host,
+                                float *lse_host, float *k_new, float *v_new, uint16_t *q,
+                                int n_q_heads, int T, int64_t n_kv, int chunk, float scale,
+                                float *out_part, float *lse_part, float *out, float *lse,
+                                kvq_stream stream)
+{
+    const char *fn = "kvq_decode_step_host";
+    if (!k_host || !v_host || !q_host || !out_host || !lse_host)
+        return set_error(KVQ_ERR_INVALID_ARG, "%s: a host buffer is NULL", fn);
+    // the device-side arguments are those of kvq_decode_step: check them all before
+    // the first copy
+    KVQ_TRY(validate_decode(layers, n_layers, q, n_q_heads, T, n_kv, chunk, scale, out_part,
+                            lse_part, fn));
+    KVQ_TRY(need(k_new, 16, "k_new", fn));
+    KVQ_TRY(need(v_new, 16, "v_new", fn));
+    const int H = layers[0].n_kv_heads, D = layers[0].head_dim;
+    const int64_t rows = (int64_t)n_layers * T * n_q_heads;
+    const int n_chunks = (int)((n_kv + chunk - 1) / chunk);
+    KVQ_TRY(validate_merge(out_part, lse_part, rows, n_chunks, D, out, lse, fn));
+    const cudaStream_t s = as_stream(stream);
+    const size_t kv_bytes = (size_t)n_layers * T * H * D * sizeof(float);
+    const struct {
+        void *dst;
+        const void *src;
+        size_t bytes;
+        const char *what;
+    } in[3] = {{q, q_host, (size_t)rows * D * sizeof(uint16_t), "q"},
+               {k_new, k_host, kv_bytes, "k"},
+               {v_new, v_host, kv_bytes, "v"}};
+    for (const auto &c : in)
+        if (cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return set_error(KVQ_ERR_COPY, "%s: host-to-device copy of %s: %s", fn, c.what,
+                             cudaGetErrorString(cudaGetLastError()));
+    KVQ_TRY(kvq_decode_step(layers, n_layers, k_new, v_new, q, n_q_heads, T, n_kv, chunk, scale,
+                            out_part, lse_part, out, lse, nullptr, 0, stream));
+    if (cudaMemcpyAsync(out_host, out, (size_t)rows * D * sizeof(float), cudaMemcpyDeviceToHost,
+                        s) != cudaSuccess ||
+        cudaMemcpyAsync(lse_host, lse, (size_t)rows * sizeof(float), cudaMemcpyDeviceToHost,
+                        s) != cudaSuccess)
+        return set_error(KVQ_ERR_COPY, "%s: device-to-host copy of the results: %s", fn,
+                         cudaGetErrorString(cudaGetLastError()));
+    return KVQ_OK;
+}
+
 kvq_status kvq_prefill_attn(const kvq_layer *layers, int n_layers, const uint16_t *q,
                             int n_q_heads, int T, int64_t n_cached, int page, float scale,
                             float *out, float *lse, float *page_out, float *page_lse,

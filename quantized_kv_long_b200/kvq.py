@@ -100,6 +100,8 @@ _SIGS = {
     "kvq_merge_lse_parts": ([_P, _P, _I32, _I64, _I32, _P, _P, _P], _I32),
     "kvq_decode_step": ([_LP, _I32, _P, _P, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P,
                          _SZ, _P], _I32),
+    "kvq_decode_step_host": ([_LP, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I64, _I32,
+                              _F32, _P, _P, _P, _P, _P], _I32),
     "kvq_prefill_attn": ([_LP, _I32, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P, _SZ,
                           _P], _I32),
     "kvq_stream_decode": ([_LP, _I32, _LP, _P, _I32, _I32, _I64, _I32, _F32, _P, _P, _P, _P, _P,
@@ -224,6 +226,19 @@ def kvq_decode_step(layers, k_new, v_new, q, n_q_heads: int, T: int, n_kv: int, 
     _check(_lib.kvq_decode_step(arr, n, _ptr(k_new), _ptr(v_new), _ptr(q), n_q_heads, T, n_kv,
                                 chunk, scale, _ptr(out_part), _ptr(lse_part), _ptr(out), _ptr(lse),
                                 _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def kvq_decode_step_host(layers, k_host, v_host, q_host, out_host, lse_host, k_new, v_new, q,
+                         n_q_heads: int, T: int, n_kv: int, chunk: int, scale: float, out_part,
+                         lse_part, out, lse, stream=None) -> None:
+    """kvq_decode_step with inputs and results in (pinned) host tensors; the device
+    tensors k_new, v_new, q, out_part, lse_part, out, lse are the copies' targets and
+    the step's buffers (see include/kvq.h)."""
+    arr, n = _layers(layers)
+    _check(_lib.kvq_decode_step_host(arr, n, _ptr(k_host), _ptr(v_host), _ptr(q_host),
+                                     _ptr(out_host), _ptr(lse_host), _ptr(k_new), _ptr(v_new),
+                                     _ptr(q), n_q_heads, T, n_kv, chunk, scale, _ptr(out_part),
+                                     _ptr(lse_part), _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def kvq_prefill_attn(layers, q, n_q_heads: int, T: int, n_cached: int, page: int, scale: float,

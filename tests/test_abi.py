@@ -258,6 +258,24 @@ def test_prefill_workspace_validation(kvq):
             ws_bytes=need)
 
 
+def test_decode_step_host_validation(kvq):
+    """kvq_decode_step_host refuses NULL host buffers and bad device arguments before
+    the first copy (nothing runs on a device here)."""
+    L = [_layer(kvq)]
+    d = dict(n_q_heads=24, T=4, n_kv=1000, chunk=1024, scale=1 / 16, out_part=A, lse_part=A,
+             out=A, lse=A)
+    host = (A, A, A, A, A)
+    dev = (A, A, A)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_decode_step_host, L, None, *host[1:], *dev,
+            **d)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_decode_step_host, L, *host[:4], None, *dev,
+            **d)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_decode_step_host, L, *host, A, A, None, **d)
+    _raises(kvq, kvq.KVQ_ERR_ALIGNMENT, kvq.kvq_decode_step_host, L, *host, A + 4, A, A, **d)
+    _raises(kvq, kvq.KVQ_ERR_INVALID_ARG, kvq.kvq_decode_step_host, L, *host, *dev,
+            **dict(d, n_kv=2000))  # beyond the capacity
+
+
 def test_cache_row_sizes_per_format(kvq):
     """Head-row bytes of each block format, as the cache helper allocates them (host
     memory here): 34, 18 and 9 bytes per 32 elements; OSCAR2 needs whole 128-element

@@ -113,3 +113,37 @@ def test_step_general_kernel_path(kvq):
     w = wl.small(wl.WORKLOADS["verify262k"], n_kv=3001)
     with kvq.test_hooks(decode_general=True):
         run_both(kvq, w, 1, 4, 3001, 512)
+
+
+def test_step_with_host_buffers_matches_device_step(kvq):
+    """kvq_decode_step_host: inputs copied from pinned host memory, results copied
+    back; the cache bytes and the host results equal the device-buffer step, bit
+    for bit, and the device buffers hold the copied inputs."""
+    w = wl.small(wl.WORKLOADS["verify262k"], n_kv=5000)
+    L, T, n_kv, chunk = 2, 4, 5000, 1024
+    cap, n0 = -(-n_kv // 8) * 8, n_kv - T
+    Hq, H, D = w.n_q_heads, w.n_kv_heads, w.head_dim
+    C = -(-n_kv // chunk)
+    ca = _cache(kvq, w, L, n0, cap)
+    cb = _cache(kvq, w, L, n0, cap)
+    k_h = torch.from_numpy(np.stack([wl.kv_rows(w, l, 0, n0, n_kv) for l in range(L)]))
+    v_h = torch.from_numpy(np.stack([wl.kv_rows(w, l, 1, n0, n_kv) for l in range(L)]))
+    q_h = torch.from_numpy(np.stack([wl.q_rows(w, l, T) for l in range(L)]))
+    op_a, lp_a, out_a, lse_a = _outputs(L, T, Hq, C, D)
+    kvq.kvq_decode_step(ca, k_h.cuda(), v_h.cuda(), q_h.cuda(), Hq, T, n_kv, chunk, w.scale,
+                        op_a, lp_a, out_a, lse_a)
+    k_pin, v_pin, q_pin = k_h.pin_memory(), v_h.pin_memory(), q_h.pin_memory()
+    out_pin = torch.full(out_a.shape, float("nan")).pin_memory()
+    lse_pin = torch.full(lse_a.shape, float("nan")).pin_memory()
+    k_d = torch.empty_like(k_h, device="cuda")
+    v_d = torch.empty_like(v_h, device="cuda")
+    q_d = torch.empty_like(q_h, device="cuda")
+    op_b, lp_b, out_b, lse_b = _outputs(L, T, Hq, C, D)
+    kvq.kvq_decode_step_host(cb, k_pin, v_pin, q_pin, out_pin, lse_pin, k_d, v_d, q_d, Hq, T,
+                             n_kv, chunk, w.scale, op_b, lp_b, out_b, lse_b)
+    kvq.kvq_check()
+    torch.cuda.synchronize()
+    for l in range(L):
+        assert torch.equal(ca.k[l], cb.k[l]) and torch.equal(ca.v[l], cb.v[l])
+    assert torch.equal(k_d.cpu(), k_h) and torch.equal(q_d.cpu(), q_h)
+    assert torch.equal(out_pin, out_a.cpu()) and torch.equal(lse_pin, lse_a.cpu())
